@@ -1,0 +1,445 @@
+"""Benchmark of the decode-time KV-cache eviction round.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload random_serving|beacon_serving|long_trace|ragged_c2|...]
+                    [--requests R] [--layers L] [--no-cpu-baseline] [--no-e2e]
+
+A step is one eviction round (kvc_update_beacons + kvc_compress for the
+beacon selector, kvc_compress for the random ones) over every (request,
+layer, KV head) segment of the workload, with the cache already resident in
+HBM.  Between steps the serving loop appends the next 64-token trigger window
+to every request (untimed), so each round sees the steady state of the
+Random Attention article's serving setup ("发现四": K=2048, 1k-token prompt,
+128 requests, compression every 64 tokens).
+
+Printed (rank 0, one JSON line): head-positions compressed per second over the
+K timed rounds (device time, CUDA events on the library's stream; max over
+ranks for N > 1), the roofline of the dominant kernel, the CPU oracle timed
+on a bounded sample (cpu_baseline), an end-to-end figure through the C ABI
+with the trigger window's K/V (and queries) read from page-locked host
+memory every step, and the clocks sampled during the timed region.
+
+Multi-GPU: one process per GPU (torchrun), each rank an independent replica
+with its own requests (the round has no exchange step: weak scaling, no
+collective on the data path; the barrier and the max-reduction of the timing
+are the only collectives).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV head-positions compressed/s per eviction round"
+UNIT = "head-positions/s"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="random_serving")
+    ap.add_argument("--selector", default=None, help="override the workload's selector")
+    ap.add_argument("--requests", type=int, default=None)
+    ap.add_argument("--layers", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--score-impl", type=int, default=0, help="beacon score kernel: 0 auto, 1 SIMT, 2 tcgen05")
+    return ap.parse_args()
+
+
+def make_workload(args):
+    from decode_kv_cache_paged_b200 import workloads as wl
+    name = args.workload
+    if name == "random_serving":
+        w = wl.random_serving()
+    elif name == "beacon_serving":
+        w = wl.beacon_serving()
+    elif name == "long_trace":
+        w = wl.long_trace()
+    elif name.startswith("ragged_c"):
+        w = wl.scaled(wl.ragged(int(name[len("ragged_c"):])), num_layers=12)
+    else:
+        raise SystemExit(f"unknown workload {name}")
+    kw = {}
+    if args.requests:
+        kw["num_requests"] = args.requests
+    if args.layers:
+        kw["num_layers"] = args.layers
+    if kw:
+        w = wl.scaled(w, **kw)
+    sel = args.selector or w.selectors[0]
+    if sel != "beacon" and w.num_beacons:
+        w = wl.scaled(w, num_beacons=0, query_window=0, num_q_heads=w.num_kv_heads)
+    return w, sel
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str):
+        self.rows = []
+        self.proc = None
+        self.idx = device_id
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[0]))
+                mx = float(r[1])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- roofline --
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "decode_kv_cache_paged_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str, units: float):
+    """DRAM bytes per launch from the committed ncu summary, scaled to `units`
+    (moved rows or keys); None if the kernel changed since the capture."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    with open(PROFILE_TRAFFIC) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash(e["sources"]):
+        return None
+    return e["dram_bytes_per_unit"] * units
+
+
+# ------------------------------------------------------------ our arm ---
+
+def run_ours(args, rank, world, dist):
+    import numpy as np
+    import torch
+
+    from decode_kv_cache_paged_b200 import workloads as wl
+    from decode_kv_cache_paged_b200 import Context, ContextSpec
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w, sel = make_workload(args)
+    w.data_seed += 7 * rank  # independent replicas
+    headroom = max(0, int(max(w.budget.max(), w.prompt.max()) + w.trigger - w.length.max()))
+    spec = ContextSpec(num_requests=w.num_requests, num_layers=w.num_layers, num_kv_heads=w.num_kv_heads,
+                       head_dim=w.head_dim, max_seq_len=w.max_seq_len(headroom),
+                       num_pages=w.pages_needed(headroom) + w.num_requests,
+                       num_q_heads=w.num_q_heads or w.num_kv_heads, num_beacons=w.num_beacons,
+                       query_window=w.query_window)
+    ctx = Context(spec, dtype=wl.torch_dtype(w.dtype), device=dev)
+    if sel == "beacon" and args.score_impl:
+        ctx.set_option(0, args.score_impl)
+    gen = wl.Generator(w, dev)
+    wl.fill(ctx, w, gen)
+    budgets = w.budget.astype(np.int32)
+    R = w.num_requests
+    ids = np.arange(R, dtype=np.int32)
+    beacon = sel == "beacon"
+    T = w.trigger
+    # trigger windows are drawn once and reused (the content does not change the cost)
+    k_win, v_win = gen.kv(R, T)
+    q_win = gen.queries(R, T) if w.query_window else None
+
+    def one_round(seed, timed):
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(ctx.stream)
+        upd_ms = ctx.update_beacons(timed=timed) if beacon else 0.0
+        st = ctx.compress(sel, budgets, seed, stats=timed)
+        ev1.record(ctx.stream)
+        return ev0, ev1, st, upd_ms
+
+    # the first compress brings the cache from its filled length to the budget;
+    # from then on every round sees L = K + trigger
+    for i in range(args.warmup):
+        if beacon:
+            ctx.update_beacons()
+        ctx.compress(sel, budgets, w.philox_seed)
+        ctx.append(ids, k_win, v_win, q_win)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clock = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    clock.start()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    rounds = []
+    for i in range(args.steps):
+        rounds.append(one_round(w.philox_seed, True))
+        ctx.append(ids, k_win, v_win, q_win)  # untimed: next trigger window
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    wall = time.perf_counter() - t_wall
+    clocks = clock.stop()
+    ms = [a.elapsed_time(b) for a, b, _, _ in rounds]
+    stats = [s for _, _, s, _ in rounds]
+    upd = [u for _, _, _, u in rounds]
+    total_ms = sum(ms)
+    if dist:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    head_pos = stats[-1]["head_positions"]
+    value = world * head_pos * args.steps / (total_ms / 1e3)
+
+    # roofline of the dominant kernel
+    peaks, peak_kind = measured_peaks()
+    sc_ms = statistics.mean(s["ms_select_compact"] for s in stats)
+    score_ms = statistics.mean(s["ms_score"] for s in stats)
+    moved = statistics.mean(s["moved_rows"] for s in stats)
+    cands = statistics.mean(s["candidates"] for s in stats)
+    rb = w.head_dim * (2 if w.dtype == "bf16" else 4)
+    # select+compact: K and V rows read and written once per moved row, the moved
+    # position entries read and written, every candidate's 4-byte key source read
+    sc_bytes = moved * (4 * rb + 8) + cands * 4
+    if beacon and score_ms > sc_ms:
+        B = w.num_beacons
+        key_bytes = statistics.mean(s["key_bytes_scored"] for s in stats)
+        keys = key_bytes / rb
+        flops = 2.0 * B * w.head_dim * (keys + cands)  # pass 1 over all keys, pass 2 over candidates
+        score_bytes = key_bytes + cands * 4 + (w.segments * B * w.head_dim * (2 if w.dtype == "bf16" else 4))
+        tc = args.score_impl == 2
+        if tc:
+            roof = {"kernel": "beacon_score_tc", "bound": "tensor", "achieved": flops / (score_ms / 1e3) / 1e12,
+                    "peak": peaks.get("bf16_tflops_sustained"), "unit": "TFLOP/s"}
+        else:
+            roof = {"kernel": "beacon_score_simt", "bound": "hbm", "achieved": score_bytes / (score_ms / 1e3) / 1e9,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        roof["traffic"] = profiled_traffic(roof["kernel"], w.name, keys)
+    else:
+        roof = {"kernel": "select_compact", "bound": "hbm", "achieved": sc_bytes / (sc_ms / 1e3) / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "traffic": profiled_traffic("select_compact", w.name, moved)}
+    roof["frac"] = roof["achieved"] / roof["peak"] if roof.get("peak") else None
+    roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})"
+    roof["algorithmic_bytes_per_launch"] = sc_bytes if roof["kernel"] == "select_compact" else None
+    roof["launch_ms"] = sc_ms if roof["kernel"] == "select_compact" else score_ms
+
+    # end to end through the C ABI: trigger window from pinned host memory,
+    # round, new lengths read back
+    e2e = None
+    if not args.no_e2e:
+        k_h = k_win.cpu().pin_memory()
+        v_h = v_win.cpu().pin_memory()
+        q_h = q_win.cpu().pin_memory() if q_win is not None else None
+        len_h = torch.empty(R, dtype=torch.int32).pin_memory()
+        lens_dev = ctx.state_tensors()["lengths"]
+        h2d = k_h.numel() * k_h.element_size() * 2 + (q_h.numel() * q_h.element_size() if q_h is not None else 0)
+        times = []
+        for i in range(args.e2e_steps + 1):
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(ctx.stream)
+            if beacon:
+                ctx.update_beacons()
+            ctx.compress(sel, budgets, w.philox_seed)
+            len_h.copy_(lens_dev, non_blocking=True)
+            ctx.append(ids, k_h, v_h, q_h)
+            b.record(ctx.stream)
+            b.synchronize()
+            if i > 0:
+                times.append(a.elapsed_time(b))
+        e2e_ms = statistics.mean(times)
+        if dist:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * head_pos / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(R * 4), "ms_per_step": e2e_ms,
+               "what": "per step: kvc_compress (+kvc_update_beacons), new lengths D2H, next trigger window's "
+                       "K/V(/queries) appended from page-locked host memory through kvc_append"}
+    ctx.sync()
+    launches = sum(s["launches"] for s in stats) + (args.steps if beacon else 0)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 (bf16 x bf16 scores)" if beacon else "u32",
+        "data": "synthetic (seeded N(0,1) K/V with 4 outlier channels x8; vMF-mixture queries)",
+        "config": {"workload": w.name, "selector": sel, "requests_per_gpu": R, "layers": w.num_layers,
+                   "kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "cache_dtype": w.dtype,
+                   "prompt": int(w.prompt[0]) if len(set(w.prompt.tolist())) == 1 else "ragged",
+                   "budget": int(w.budget[0]) if len(set(w.budget.tolist())) == 1 else "ragged",
+                   "trigger": T, "beacons": w.num_beacons, "page_size": 16,
+                   "head_positions_per_round_per_gpu": head_pos,
+                   "parallelism": f"replicas x{world} (no collective on the data path)",
+                   "l2": "inputs larger than L2: the cache is tens of GB vs 126 MB L2, and each "
+                         "trigger append between rounds writes >1 GB"},
+        "roofline": roof,
+        "phases_ms": {"select_compact": sc_ms, "score": score_ms, "update": statistics.mean(upd) if beacon else 0.0},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "wall_s_timed_region": wall,
+    }
+    return out, w, sel
+
+
+# ------------------------------------------------------- oracle timing ---
+
+def oracle_sample_rate(w, sel, budget_s: float, rank_seed: int = 0):
+    """Times the oracle (single thread) on whole segments of the workload until
+    ~budget_s seconds of oracle time; returns (head_positions/s, description)."""
+    import numpy as np
+
+    import oracle
+    rng = np.random.default_rng(1234 + rank_seed)
+    d = w.head_dim
+    es = 2 if w.dtype == "bf16" else 4
+    t_total = 0.0
+    hp = 0
+    n_seg = 0
+    H, Ly = w.num_kv_heads, w.num_layers
+    segs = [(r, l, h) for r in range(w.num_requests) for l in range(Ly) for h in range(H)]
+    cache = {}
+    while t_total < budget_s and n_seg < len(segs):
+        r, l, h = segs[n_seg]
+        L, P, K = int(w.length[r]), int(w.prompt[r]), int(w.budget[r])
+        key = (L, P)
+        if key not in cache:
+            rows_k = rng.integers(0, 255, (L, d * es), dtype=np.uint8)
+            rows_v = rng.integers(0, 255, (L, d * es), dtype=np.uint8)
+            keys = rng.standard_normal((L, d)) if sel == "beacon" else None
+            pts = rng.standard_normal((w.query_window * w.G, d)) if sel == "beacon" else None
+            cache[key] = (rows_k, rows_v, keys, pts)
+        rows_k, rows_v, keys, pts = cache[key]
+        pos = np.arange(L, dtype=np.int32)
+        t0 = time.perf_counter()
+        if sel == "beacon":
+            c, cnt, _ = oracle.beacon_update(pts, np.zeros((w.num_beacons, d)), np.zeros(w.num_beacons), init=True)
+            kept, _ = oracle.beacon_round_segment(keys, P, K, oracle.round_bf16(c) if w.dtype == "bf16" else c)
+        else:
+            kept, _ = oracle.random_round_segment(w.philox_seed, 0, r, l, h, sel == "random_shared", P, K, pos)
+        oracle.compact_rows(rows_k, P, kept[P:])
+        oracle.compact_rows(rows_v, P, kept[P:])
+        t_total += time.perf_counter() - t0
+        hp += L
+        n_seg += 1
+    desc = (f"{n_seg} whole segments (requests from 0, all layers and heads in order) of {w.name}, "
+            f"selector {sel}: score + full-sort select + K/V compaction, {t_total:.1f} s of oracle time")
+    return hp / t_total, desc, n_seg
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, on the host cores."""
+    w, sel = make_workload(args)
+    per_step = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, sel, per_step / 4)
+    rates = []
+    desc = ""
+    for s in range(args.steps):
+        rate, desc, _ = oracle_sample_rate(w, sel, per_step, rank_seed=s)
+        rates.append(rate)
+    value = statistics.mean(rates)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.head_positions / value * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "selector": sel},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        out, w, sel = run_ours(args, rank, world, dist)
+        if rank == 0:
+            if not args.no_cpu_baseline:
+                rate, desc, _ = oracle_sample_rate(w, sel, 12.0)
+                out["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+            print(json.dumps(out), flush=True)
+    finally:
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

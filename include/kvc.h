@@ -119,7 +119,7 @@ typedef struct {
   float ms_score;                /* device time of the beacon scoring kernel(s) */
   float ms_select_compact;       /* device time of the fused select + compaction kernel */
   float ms_total;                /* device time of the whole call */
-  float reserved;
+  int32_t launches;              /* kernels this call launched */
 } kvc_round_stats;
 
 /* Zero-copy view of the context's device state (pointers into the pools and

@@ -1,0 +1,159 @@
+"""BeaconKV update and scoring on the GPU against the oracle.
+
+Staged parity: the oracle's beacon update is compared assignment by
+assignment (exact, or a counted near-tie), then recomputed from the GPU's
+assignments (fp32 vs double running means); the oracle's scores are computed
+from the GPU's scoring copy of the beacons and the pre-round keys, then
+compared within |g - o| <= 1e-5 + 1e-3|o|; the kept set must match the
+oracle's except within 1e-4 of the threshold, with equal counts."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from decode_kv_cache_paged_b200 import workloads as wl
+from gpu_helpers import band_check, check_scores, dense_layer, make_context
+
+pytestmark = pytest.mark.gpu
+
+
+def _fill_recording(ctx, w, gen):
+    """Fill like workloads.fill, keeping the queries of the last W steps per request."""
+    R = w.num_requests
+    W = w.query_window
+    qwin = {}
+    for r in range(R):
+        P, L = int(w.prompt[r]), int(w.length[r])
+        ids = np.array([r], np.int32)
+        done = 0
+        while done < P:
+            T = min(256, P - done)
+            k, v = gen.kv(1, T)
+            ctx.append(ids, k, v, None, protect=True)
+            done += T
+        q_from = L - min(W, L - P)
+        qs = []
+        while done < L:
+            T = min(256 if done < q_from else 16, (q_from if done < q_from else L) - done)
+            k, v = gen.kv(1, T)
+            q = gen.queries(1, T) if done >= q_from else None
+            ctx.append(ids, k, v, q)
+            if q is not None:
+                qs.append(q[0].float().cpu().numpy().astype(np.float64))  # [Ly, T, Hq, d]
+            done += T
+        qwin[r] = np.concatenate(qs, axis=1)[:, -W:]  # [Ly, steps, Hq, d]
+    return qwin
+
+
+def run_beacon(w, sample=None, score_impl=None):
+    ctx = make_context(w)
+    if score_impl is not None:
+        ctx.set_option(0, score_impl)
+    gen = wl.Generator(w, "cuda")
+    qwin = _fill_recording(ctx, w, gen)
+    R, Ly, H, d, B, G = w.num_requests, w.num_layers, w.num_kv_heads, w.head_dim, w.num_beacons, w.G
+    W = w.query_window
+    assign = torch.full((R, Ly, H, W * G), -1, dtype=torch.int32, device="cuda")
+    ctx.update_beacons(assign_out=assign)
+    ctx.sync()
+    st = ctx.state_tensors()
+    g_beacons = st["beacons"].cpu().numpy().astype(np.float64)
+    g_scoring = st["beacons_scoring"].float().cpu().numpy().astype(np.float64)
+    g_counts = st["beacon_counts"].cpu().numpy()
+    g_assign = assign.cpu().numpy()
+    # the scoring copy is the fp32 beacon rounded to the cache dtype (torch's RNE cast)
+    assert torch.equal(st["beacons_scoring"], st["beacons"].to(ctx.dtype))
+    segs = [(r, l, h) for r in range(R) for l in range(Ly) for h in range(H)]
+    if sample is not None:
+        segs = [segs[i] for i in np.random.default_rng(0).choice(len(segs), sample, replace=False)]
+    near_ties = 0
+    for (r, l, h) in segs:
+        pts = oracle.segment_points(qwin[r][l], h, G)
+        n = len(pts)
+        ga = g_assign[r, l, h, :n]
+        c_o, cnt_o, a_o = oracle.beacon_update(pts, np.zeros((B, d)), np.zeros(B), init=True)
+        if not np.array_equal(a_o, ga):
+            # differing assignments must be near-ties of the squared distance
+            c0 = pts[(np.arange(B) * n) // B]
+            for p in np.nonzero(a_o != ga)[0]:
+                d_o = np.sum((pts[p] - c0[a_o[p]]) ** 2)
+                d_g = np.sum((pts[p] - c0[ga[p]]) ** 2)
+                assert abs(d_o - d_g) <= 1e-5 * max(d_o, 1e-30), (r, l, h, p, d_o, d_g)
+                near_ties += 1
+        c_s, cnt_s, _ = oracle.beacon_update(pts, np.zeros((B, d)), np.zeros(B), init=True, assign_override=ga)
+        assert np.array_equal(cnt_s, g_counts[r, l, h])
+        assert np.allclose(g_beacons[r, l, h], c_s, rtol=1e-5, atol=1e-6), (r, l, h)
+    # the round
+    lengths, prompts = ctx.lengths()
+    cap = int(lengths.max())
+    need_l = sorted({l for (_, l, _) in segs})
+    pre = {l: dense_layer(ctx, l, range(R), cap, lengths, with_kv=True) if sample is None else None
+           for l in need_l}
+    if sample is not None:
+        # only the sampled (request, layer) pairs, to bound device memory
+        for l in need_l:
+            rs = sorted({r for (r, ll, _) in segs if ll == l})
+            pos, k, v = dense_layer(ctx, l, rs, cap, lengths, with_kv=True)
+            full_pos = np.full((R,) + pos.shape[1:], -1, np.int64)
+            full_k = torch.zeros((R,) + tuple(k.shape[1:]), dtype=k.dtype, device=k.device)
+            full_v = torch.zeros_like(full_k)
+            idx = torch.as_tensor(rs, device=k.device)
+            full_pos[rs] = pos
+            full_k[idx] = k
+            full_v[idx] = v
+            pre[l] = (full_pos, full_k, full_v)
+    scores = torch.zeros((R, Ly, H, ctx.spec.max_seq_len), dtype=torch.float32, device="cuda")
+    budgets = w.budget.astype(np.int32)
+    stats = ctx.compress("beacon", budgets, w.philox_seed, debug_scores=scores, stats=True)
+    ctx.sync()
+    new_len, _ = ctx.lengths()
+    g_scores = scores.cpu().numpy()
+    max_rel = 0.0
+    differ = in_abs = in_rel = 0
+    for (r, l, h) in segs:
+        L, P, K = int(lengths[r]), int(prompts[r]), int(budgets[r])
+        keys = pre[l][1][r, h, :L].float().cpu().numpy().astype(np.float64)
+        o_sc, _ = oracle.beacon_score(keys, g_scoring[r, l, h], P)
+        if L <= K:
+            continue
+        N, M = L - P, max(0, K - P)
+        assert new_len[r] == P + M
+        if M == 0:
+            continue
+        max_rel = max(max_rel, check_scores(g_scores[r, l, h, :N], o_sc))
+        post_pos, post_k, post_v = dense_layer(ctx, l, [r], int(new_len[r]), new_len, with_kv=True)
+        gpu_kept = np.searchsorted(pre[l][0][r, h, :L], post_pos[0, h])
+        assert np.array_equal(pre[l][0][r, h, gpu_kept], post_pos[0, h])
+        assert np.array_equal(gpu_kept[:P], np.arange(P))
+        dd, ia, ir = band_check(gpu_kept[P:], o_sc, P, M, N)
+        differ += dd
+        in_abs += ia
+        in_rel += ir
+        # compacted bytes follow the GPU's own selection exactly
+        ks = torch.as_tensor(gpu_kept, device="cuda")
+        assert torch.equal(post_k[0, h], pre[l][1][r, h, ks])
+        assert torch.equal(post_v[0, h], pre[l][2][r, h, ks])
+    ctx.close()
+    return {"near_tie_assignments": near_ties, "max_rel_score_err": max_rel, "index_differ": differ,
+            "in_band_abs": in_abs, "in_band_rel": in_rel, "stats": stats}
+
+
+def test_tiny_beacon():
+    out = run_beacon(wl.tiny())
+    assert out["index_differ"] == 0
+
+
+def test_beacon_serving_small():
+    out = run_beacon(wl.beacon_serving(R=3, layers=2))
+    print(out)
+
+
+def test_beacon_serving_full_size_sampled():
+    out = run_beacon(wl.beacon_serving(), sample=24)
+    print(out)
+
+
+def test_long_trace_sampled():
+    w = wl.scaled(wl.long_trace(), num_requests=2, num_layers=4)
+    out = run_beacon(w, sample=3)
+    print(out)
