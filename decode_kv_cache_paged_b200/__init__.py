@@ -101,6 +101,7 @@ _SIGS = {
     "kvc_sync": (_i32, [_P]),
     "kvc_status_string": (ctypes.c_char_p, [_i32]),
     "kvc_last_error": (ctypes.c_char_p, [_P]),
+    "kvc_beacon_select_noalloc": (_i32, [_P, _P, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)

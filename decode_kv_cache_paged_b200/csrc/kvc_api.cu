@@ -92,6 +92,11 @@ Layout make_layout(const kvc_config &c) {
 
 }  // namespace
 
+namespace kvc {
+// Message for kvc_last_error(NULL) from entry points that take no context.
+void set_thread_error(const std::string &msg) { g_create_error = msg; }
+}  // namespace kvc
+
 struct kvc_ctx {
   kvc_config cfg{};
   Layout lay{};

@@ -243,6 +243,43 @@ kvc_status kvc_sync(kvc_ctx *ctx);
 const char *kvc_status_string(kvc_status s);
 const char *kvc_last_error(const kvc_ctx *ctx);
 
+/* Allocation-free beacon score and top-K selection of S dense segments.
+ * The pages have no counterpart: this entry point exists for callers that
+ * cannot allocate device memory, such as code running while a CUDA graph is
+ * captured (cudaMalloc is not allowed there), plug-ins confined to another
+ * engine's fixed memory arena, or hosts with no device allocator, and which
+ * therefore cannot give kvc_create a workspace.  It needs no context.
+ *   keys:    device [S][L][head_dim] dtype, each segment's cached keys in
+ *            position order (the prompt first).
+ *   beacons: device [S][B][head_dim] dtype, each segment's beacon scoring copies.
+ *   P, K:    protected prompt length and budget, shared by the S segments.
+ *   kept_out:   device int32 [S][R], R = L if L <= K, else max(P, K): the kept
+ *               slots of each segment, ascending (the prompt, then the best
+ *               max(0, K-P) candidates by (score desc, slot asc)).
+ *   scores_out: device float [S][L-P] or NULL; when the round evicts some but
+ *               not all candidates it receives each candidate's score, else it
+ *               is left untouched.
+ *   cuda_stream: cudaStream_t on the inputs' device (NULL = legacy stream).
+ * The scores and the selection are those of kvc_compress(KVC_SEL_BEACON)
+ * for the same keys and beacons.  Scratch: the scores pass between the two
+ * kernels through a fixed array of 1,048,576 floats (4 MiB) in the library's
+ * device memory, held on every GPU that loads the library until the process
+ * exits; S*(L-P) above 1,048,576 is rejected with KVC_ERR_INVALID_ARG.  No
+ * part of the array needs to start at zero: each call writes every score it
+ * reads.  All calls on a device share that device's array, which keeps the
+ * last call's contents, so calls that overlap on the same GPU (for example on
+ * two streams) race on it: serialise them.  The first
+ * call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * which may load the library's kernels); make that first call before any
+ * stream capture.  The call allocates nothing: no cudaMalloc, cudaFree or
+ * allocating library routine.  Limits: L <= 32768, B in [1, 256], head_dim 64
+ * or 128.  Errors: KVC_ERR_INVALID_ARG (message in kvc_last_error(NULL)),
+ * KVC_ERR_CUDA. */
+kvc_status kvc_beacon_select_noalloc(const void *keys, const void *beacons, int32_t S, int32_t L,
+                                     int32_t P, int32_t K, int32_t B, int32_t head_dim,
+                                     int32_t dtype, int32_t *kept_out, float *scores_out,
+                                     void *cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif
