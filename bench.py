@@ -47,7 +47,7 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="random_serving")
@@ -61,8 +61,20 @@ def parse():
     return ap.parse_args()
 
 
+def load_workloads():
+    """The seeded workload generators (workloads.py), loaded by path so that the
+    reference arm does not load libkvc.so."""
+    import importlib.util
+    path = os.path.join(ROOT, "decode_kv_cache_paged_b200", "workloads.py")
+    spec = importlib.util.spec_from_file_location("kvc_workloads", path)
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules["kvc_workloads"] = mod
+    spec.loader.exec_module(mod)
+    return mod
+
+
 def make_workload(args):
-    from decode_kv_cache_paged_b200 import workloads as wl
+    wl = load_workloads()
     name = args.workload
     if name == "random_serving":
         w = wl.random_serving()
@@ -90,7 +102,7 @@ def make_workload(args):
 # ---------------------------------------------------------------- clocks --
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -105,7 +117,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
@@ -174,6 +186,58 @@ def profiled_traffic(kernel: str, workload: str, units: float):
 
 # ------------------------------------------------------------ our arm ---
 
+def aggregate(local_ms: float, units_per_rank: float, steps: int, world: int, dist, device=None):
+    """Whole-job throughput: units all ranks processed / the slowest rank's time."""
+    total_ms = local_ms
+    if dist is not None and world > 1:
+        import torch
+        t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    return world * units_per_rank * steps / (total_ms / 1e3), total_ms
+
+
+class Refill:
+    """Brings every request back to its pre-round length between rounds
+    (untimed): the next 64-token trigger window for the serving workloads
+    (drawn once and reused), freshly drawn tokens for the others."""
+
+    def __init__(self, ctx, w, gen):
+        import numpy as np
+        self.ctx, self.w, self.gen = ctx, w, gen
+        self.np = np
+        self.window = None
+        if len(set(w.length.tolist())) == 1 and len(set(w.budget.tolist())) == 1 and \
+                int(w.length[0]) - max(int(w.budget[0]), int(w.prompt[0])) == w.trigger:
+            R = w.num_requests
+            k, v = gen.kv(R, w.trigger)
+            q = gen.queries(R, w.trigger) if w.query_window else None
+            self.window = (np.arange(R, dtype=np.int32), k, v, q)
+
+    def __call__(self):
+        np, w, ctx = self.np, self.w, self.ctx
+        if self.window is not None:
+            ln, _ = ctx.lengths()
+            if np.all(ln + w.trigger == w.length):
+                ctx.append(*self.window)
+                return
+        ln, _ = ctx.lengths()
+        need = w.length - ln
+        groups = {}
+        for r in range(w.num_requests):
+            if need[r] > 0:
+                groups.setdefault(int(need[r]), []).append(r)
+        for T_all, reqs in groups.items():
+            ids = np.array(reqs, np.int32)
+            done = 0
+            q_from = T_all - min(w.query_window, T_all) if w.query_window else T_all
+            while done < T_all:
+                T = min(256 if done < q_from else 16, (q_from if done < q_from else T_all) - done)
+                k, v = self.gen.kv(len(ids), T)
+                q = self.gen.queries(len(ids), T) if done >= q_from else None
+                ctx.append(ids, k, v, q)
+                done += T
+
 def run_ours(args, rank, world, dist):
     import numpy as np
     import torch
@@ -202,9 +266,7 @@ def run_ours(args, rank, world, dist):
     ids = np.arange(R, dtype=np.int32)
     beacon = sel == "beacon"
     T = w.trigger
-    # trigger windows are drawn once and reused (the content does not change the cost)
-    k_win, v_win = gen.kv(R, T)
-    q_win = gen.queries(R, T) if w.query_window else None
+    refill = Refill(ctx, w, gen)
 
     def one_round(seed, timed):
         ev0 = torch.cuda.Event(enable_timing=True)
@@ -221,7 +283,7 @@ def run_ours(args, rank, world, dist):
         if beacon:
             ctx.update_beacons()
         ctx.compress(sel, budgets, w.philox_seed)
-        ctx.append(ids, k_win, v_win, q_win)
+        refill()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -233,7 +295,7 @@ def run_ours(args, rank, world, dist):
     rounds = []
     for i in range(args.steps):
         rounds.append(one_round(w.philox_seed, True))
-        ctx.append(ids, k_win, v_win, q_win)  # untimed: next trigger window
+        refill()  # untimed: back to the pre-round lengths
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -242,13 +304,8 @@ def run_ours(args, rank, world, dist):
     ms = [a.elapsed_time(b) for a, b, _, _ in rounds]
     stats = [s for _, _, s, _ in rounds]
     upd = [u for _, _, _, u in rounds]
-    total_ms = sum(ms)
-    if dist:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
     head_pos = stats[-1]["head_positions"]
-    value = world * head_pos * args.steps / (total_ms / 1e3)
+    value, total_ms = aggregate(sum(ms), head_pos, args.steps, world, dist, dev)
 
     # roofline of the dominant kernel
     peaks, peak_kind = measured_peaks()
@@ -266,13 +323,16 @@ def run_ours(args, rank, world, dist):
         keys = key_bytes / rb
         flops = 2.0 * B * w.head_dim * (keys + cands)  # pass 1 over all keys, pass 2 over candidates
         score_bytes = key_bytes + cands * 4 + (w.segments * B * w.head_dim * (2 if w.dtype == "bf16" else 4))
-        tc = args.score_impl == 2
+        tc = stats[-1].get("score_impl", 0) == 2 or args.score_impl == 2
         if tc:
             roof = {"kernel": "beacon_score_tc", "bound": "tensor", "achieved": flops / (score_ms / 1e3) / 1e12,
-                    "peak": peaks.get("bf16_tflops_sustained"), "unit": "TFLOP/s"}
+                    "peak": peaks.get("bf16_tflops_sustained"), "unit": "TFLOP/s",
+                    "hbm_gbs": score_bytes / (score_ms / 1e3) / 1e9}
         else:
-            roof = {"kernel": "beacon_score_simt", "bound": "hbm", "achieved": score_bytes / (score_ms / 1e3) / 1e9,
-                    "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+            # SIMT fp32: 148 SMs x 128 FP32 lanes x 2 flop per FMA x the max SM clock
+            simt_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+            roof = {"kernel": "beacon_score_simt", "bound": "alu", "achieved": flops / (score_ms / 1e3) / 1e12,
+                    "peak": simt_peak, "unit": "TFLOP/s", "hbm_gbs": score_bytes / (score_ms / 1e3) / 1e9}
         roof["traffic"] = profiled_traffic(roof["kernel"], w.name, keys)
     else:
         roof = {"kernel": "select_compact", "bound": "hbm", "achieved": sc_bytes / (sc_ms / 1e3) / 1e9,
@@ -286,7 +346,8 @@ def run_ours(args, rank, world, dist):
     # end to end through the C ABI: trigger window from pinned host memory,
     # round, new lengths read back
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and refill.window is not None:
+        _, k_win, v_win, q_win = refill.window
         k_h = k_win.cpu().pin_memory()
         v_h = v_win.cpu().pin_memory()
         q_h = q_win.cpu().pin_memory() if q_win is not None else None
@@ -308,12 +369,8 @@ def run_ours(args, rank, world, dist):
             b.synchronize()
             if i > 0:
                 times.append(a.elapsed_time(b))
-        e2e_ms = statistics.mean(times)
-        if dist:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * head_pos / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+        e2e_value, e2e_ms = aggregate(statistics.mean(times), head_pos, 1, world, dist, dev)
+        e2e = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(R * 4), "ms_per_step": e2e_ms,
                "what": "per step: kvc_compress (+kvc_update_beacons), new lengths D2H, next trigger window's "
                        "K/V(/queries) appended from page-locked host memory through kvc_append"}
