@@ -323,7 +323,7 @@ def run_ours(args, rank, world, dist):
         keys = key_bytes / rb
         flops = 2.0 * B * w.head_dim * (keys + cands)  # pass 1 over all keys, pass 2 over candidates
         score_bytes = key_bytes + cands * 4 + (w.segments * B * w.head_dim * (2 if w.dtype == "bf16" else 4))
-        tc = stats[-1].get("score_impl", 0) == 2 or args.score_impl == 2
+        tc = stats[-1].get("score_kernel", 0) == 2
         if tc:
             roof = {"kernel": "beacon_score_tc", "bound": "tensor", "achieved": flops / (score_ms / 1e3) / 1e12,
                     "peak": peaks.get("bf16_tflops_sustained"), "unit": "TFLOP/s",

@@ -68,10 +68,11 @@ class kvc_round_stats(ctypes.Structure):
                 ("evicted", ctypes.c_int64), ("moved_rows", ctypes.c_int64),
                 ("compaction_bytes", ctypes.c_int64), ("key_bytes_scored", ctypes.c_int64),
                 ("ms_score", ctypes.c_float), ("ms_select_compact", ctypes.c_float),
-                ("ms_total", ctypes.c_float), ("launches", ctypes.c_int32)]
+                ("ms_total", ctypes.c_float), ("launches", ctypes.c_int32),
+                ("score_kernel", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
     def as_dict(self):
-        return {f: getattr(self, f) for f, _ in self._fields_}
+        return {f: getattr(self, f) for f, _ in self._fields_ if f != "reserved"}
 
 
 class kvc_view(ctypes.Structure):

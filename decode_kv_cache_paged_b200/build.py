@@ -26,6 +26,11 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-re
          "-I" + os.path.join(ROOT, "include")]
 
 
+# Extra flags per source.  The tensor-core beacon score flushes fp32 denormals
+# (its exp2 terms below 2^-126 are negligible next to the sum they join).
+EXTRA = {"beacon_score_tc.cu": ["-ftz=true"]}
+
+
 def _sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
@@ -52,7 +57,8 @@ def build(verbose: bool = False, force: bool = False, ptxas_verbose: bool = Fals
         o = os.path.join(BUILD, os.path.basename(s)[:-3] + ".o")
         objs.append(o)
         if force or _stale(o, [s] + hdrs):
-            cmd = [NVCC] + ARCH + FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", s, "-o", o]
+            cmd = [NVCC] + ARCH + FLAGS + EXTRA.get(os.path.basename(s), []) + \
+                (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", s, "-o", o]
             jobs.append(cmd)
 
     def run(cmd):

@@ -1,24 +1,553 @@
-// beacon_score_tc.cu -- tcgen05 (5th-generation tensor core) beacon score for
-// bf16 caches.  Placeholder until the tensor-core kernel lands: reports
-// "not supported" so the SIMT kernel serves every case.
+// beacon_score_tc.cu -- BeaconKV beacon score on the 5th-generation tensor
+// cores (tcgen05) for bf16 caches with head_dim 128.
+//
+// Score (the library's definition; the BeaconKV explainer, §3.2, leaves the
+// importance rule open): z_bj = c_b.k_j/sqrt(d), lse_b = log sum_j exp(z_bj)
+// over every cached key j < L, score_j = max_b exp(z_bj - lse_b) for the
+// generated keys j in [P, L).  The contraction c_b.k_j is bf16 x bf16 with
+// fp32 accumulation; with 64+ beacons it carries 64+ flop per key byte, above
+// what the SIMT pipes sustain at HBM speed, so it runs on tcgen05.mma with
+// the accumulators in tensor memory (TMEM).
+//
+// Structure: a persistent kernel, one CTA per SM, walking its segments
+// (request, layer, KV head) and, per segment, the 128-key tiles of the key
+// sequence twice:
+//   pass 1 (all tiles): D1[b, j] = C K^T with the beacons on TMEM lanes
+//          (A = beacons, M = 128 rows per MMA, two MMAs for B > 128) and 128
+//          keys on columns; each epilogue thread owns one beacon row and keeps
+//          an online (max, sum of 2^u) over its columns;
+//   pass 2 (tiles holding generated keys): D2[j, b] = K C^T with the keys on
+//          lanes (A = keys, M = 128, N = B); each epilogue thread owns one key
+//          and takes the max over beacon columns of u_bj - lse2_b.
+// Work in base 2: u = z_raw * log2(e)/sqrt(d), lse2 = log2 sum 2^u, score =
+// 2^(max_b u_bj - lse2_b).
+// Warp roles: warp 0 allocates TMEM and issues the TMA loads (one 2-D tiled
+// load per (page, 64-column half): a page holds 16 keys x 256 B contiguous,
+// the tensor map covers the whole pool as rows of 128 bf16, 128-byte
+// swizzle); warp 1 issues the MMAs (one elected lane) and commits them to
+// mbarriers; warps 2-5 run the epilogue (tcgen05.ld of 64 columns at a time;
+// sums and maxima in 8 independent partials to keep the pipes busy).
+// Key tiles rotate through 4 shared-memory stages; the accumulators through
+// two 256-column TMEM buffers.  No load uses cluster multicast.
+// Every mbarrier wait is bounded (2 s of %globaltimer): on expiry the kernel
+// records KVC_ERR_DEVICE_TIMEOUT in the status word, the other roles see the
+// abort flag and leave, and TMEM is released before the CTA exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "kvc_internal.h"
 
 namespace kvc {
+namespace {
 
-bool beacon_score_tc_supported(int d, int B, int dtype) {
-  (void)d;
-  (void)B;
-  (void)dtype;
-  return false;
+constexpr int kTileKeys = 128;
+constexpr int kStages = 4;
+constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
+
+struct TcParams {
+  const int32_t *block_table;
+  const SegDesc *segs;
+  float *scores;
+  float *lse_out;
+  int32_t *status;
+  int64_t num_pages;
+  int32_t bt_stride, layers, hkv, B, max_seq, n_segs;
+  float alpha;  // log2(e) / sqrt(d)
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// One try: the thread may be suspended until the phase completes or up to
+// the hint (1 ms) elapses, so waiting warps do not spin on issue slots.
+__device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait by lane 0 only, result broadcast: keeps the warp converged.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *status);
+// Bounded wait for the phase of `parity` to complete; false on timeout/abort.
+// With honor_abort false (clean-up of copies and MMAs in flight) only the
+// time limit ends the wait.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *status, bool honor_abort = true) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try(bar, parity)) return true;
+    if (honor_abort && *abort_flag) return false;
+    if (global_ns() - t0 > kWaitNs) {
+      atomicCAS(status, kDevOk, kDevTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *status) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+// K-major operand in the canonical 128-byte-swizzled layout: 8-row atoms of
+// 128 B, atoms 1024 B apart (SBO); the K offset inside an atom is added to the
+// start address.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;             // leading byte offset (unused with swizzle)
+  d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset: 8 rows x 128 B
+  d |= (uint64_t)1 << 46;             // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;             // 128-byte swizzle
+  return d;
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0));
+}
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]),
+        "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]),
+        "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+        "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]),
+        "=r"(r[63])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+// Per-segment geometry shared by every role.
+struct SegGeom {
+  int r, l, h, L, P;
+  int64_t seg_flat;
+  int n1, t2, n2;  // pass-1 tiles, first pass-2 tile, pass-2 tiles
+};
+__device__ __forceinline__ SegGeom seg_geom(const TcParams &p, int s) {
+  SegGeom g;
+  g.h = s % p.hkv;
+  g.l = (s / p.hkv) % p.layers;
+  const SegDesc sd = p.segs[s / (p.hkv * p.layers)];
+  g.r = sd.req;
+  g.L = sd.L;
+  g.P = sd.P;
+  g.seg_flat = ((int64_t)g.r * p.layers + g.l) * p.hkv + g.h;
+  g.n1 = (g.L + kTileKeys - 1) / kTileKeys;
+  g.t2 = g.P / kTileKeys;
+  g.n2 = g.n1 - g.t2;
+  return g;
 }
 
-cudaError_t launch_beacon_score_tc(const BeaconScoreParams &p, int n_req, int max_l,
-                                   cudaStream_t s) {
-  (void)p;
-  (void)n_req;
+template <int CROWS, int NCB>
+__global__ void __launch_bounds__(kThreads, 1)
+    beacon_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap cmap,
+                           TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr uint32_t kCBytes = CROWS * 256;          // beacon tile: CROWS rows x 128 bf16
+  constexpr uint32_t kTileBytes = kTileKeys * 256;   // 32 KB
+  uint8_t *cbuf = smem;                              // [NCB][2 K-halves][CROWS][128 B]
+  uint8_t *kbuf = smem + NCB * kCBytes;              // [kStages][2][128][128 B]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(kbuf + kStages * kTileBytes);
+  uint64_t *full = bars, *empty = bars + kStages;
+  uint64_t *acc_full = bars + 2 * kStages, *acc_empty = acc_full + 2;
+  uint64_t *c_full = acc_empty + 2, *c_empty = c_full + 2, *mma_done = c_empty + 2;
+  uint64_t *epi_bar = mma_done + 1;  // the 4 epilogue warps, once per segment
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(epi_bar + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  float *lse2 = reinterpret_cast<float *>(tmem_slot + 4);  // [2][256]
+  float *part = lse2 + 512;                                 // [2][64] (m, sum) of the upper copy
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+      mbar_init(&c_full[i], 1);
+      mbar_init(&c_empty[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    mbar_init(epi_bar, 4);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int B = p.B;
+  // With 64 beacons or fewer the tile holds two copies of them (rows 0-63 and
+  // 64-127) so that all four epilogue warps share pass 1, each copy taking
+  // half of the key columns.
+  const bool dup = B <= 64;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;  // key-tile counter across segments
+      int si = 0;       // local segment counter
+      for (int s = blockIdx.x; s < p.n_segs && !*abort_flag; s += gridDim.x, ++si) {
+        const SegGeom g = seg_geom(p, s);
+        const int cb = si % NCB;
+        if (!mbar_wait(&c_empty[cb], ((si / NCB) & 1) ^ 1, abort_flag, p.status)) break;
+        mbar_expect_tx(&c_full[cb], (uint32_t)B * 256u * (dup ? 2u : 1u));
+        const int crow = (int)(g.seg_flat * B);
+        for (int copy = 0; copy < (dup ? 2 : 1); ++copy) {
+          uint8_t *cdst = cbuf + cb * kCBytes + copy * 64 * 128;
+          tma_load_2d(smem_u32(cdst), &cmap, 0, crow, &c_full[cb]);
+          tma_load_2d(smem_u32(cdst + CROWS * 128), &cmap, 64, crow, &c_full[cb]);
+        }
+        const int32_t *bt = p.block_table + (int64_t)g.r * p.bt_stride;
+        const int pages = (g.L + kPage - 1) / kPage;
+        for (int t = 0; t < g.n1 + g.n2 && !*abort_flag; ++t, ++it) {
+          const int tile = t < g.n1 ? t : g.t2 + (t - g.n1);
+          const int st = it % kStages;
+          if (!mbar_wait(&empty[st], ((it / kStages) & 1) ^ 1, abort_flag, p.status)) break;
+          const int pg0 = tile * (kTileKeys / kPage);
+          const int npg = min(kTileKeys / kPage, pages - pg0);
+          mbar_expect_tx(&full[st], (uint32_t)npg * 2u * 2048u);
+          uint8_t *dst = kbuf + st * kTileBytes;
+          for (int q = 0; q < npg; ++q) {
+            const int64_t row = (((int64_t)g.l * p.num_pages + bt[pg0 + q]) * p.hkv + g.h) * kPage;
+            tma_load_2d(smem_u32(dst + q * 2048), &kmap, 0, (int)row, &full[st]);
+            tma_load_2d(smem_u32(dst + kTileKeys * 128 + q * 2048), &kmap, 64, (int)row, &full[st]);
+          }
+        }
+      }
+      if (*abort_flag) {
+        // let loads already issued land before the CTA's shared memory goes away
+        for (int i = 0; i < kStages && it > 0; ++i) {
+          const uint32_t k = it - 1 - i;
+          mbar_wait(&full[k % kStages], (k / kStages) & 1, abort_flag, p.status, false);
+          if (k == 0) break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, acc_it = 0;
+      int si = 0;
+      const uint32_t idesc1 = idesc_bf16_f32(128, kTileKeys);
+      const uint32_t idesc2 = idesc_bf16_f32(128, B);
+      bool ok = true;
+      for (int s = blockIdx.x; s < p.n_segs && ok; s += gridDim.x, ++si) {
+        const SegGeom g = seg_geom(p, s);
+        const int cb = si % NCB;
+        ok = mbar_wait(&c_full[cb], (si / NCB) & 1, abort_flag, p.status);
+        if (!ok) break;
+        const uint32_t c_addr = smem_u32(cbuf + cb * kCBytes);
+        for (int t = 0; t < g.n1 + g.n2; ++t, ++it, ++acc_it) {
+          const int st = it % kStages, buf = acc_it & 1;
+          ok = mbar_wait(&full[st], (it / kStages) & 1, abort_flag, p.status) &&
+               mbar_wait(&acc_empty[buf], ((acc_it >> 1) & 1) ^ 1, abort_flag, p.status);
+          if (!ok) break;
+          tmem_fence_after();
+          const uint32_t k_addr = smem_u32(kbuf + st * kTileBytes);
+          const uint32_t d = tmem_base + buf * 256;
+          if (t < g.n1) {
+            for (int half = 0; half * 128 < B; ++half)
+              for (int kb = 0; kb < 2; ++kb)
+                for (int ks = 0; ks < 4; ++ks) {
+                  const uint64_t a = sw128_desc(c_addr + kb * CROWS * 128 + half * 128 * 128 + ks * 32);
+                  const uint64_t b = sw128_desc(k_addr + kb * kTileKeys * 128 + ks * 32);
+                  umma(d + half * 128, a, b, idesc1, (kb | ks) != 0);
+                }
+          } else {
+            for (int kb = 0; kb < 2; ++kb)
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t a = sw128_desc(k_addr + kb * kTileKeys * 128 + ks * 32);
+                const uint64_t b = sw128_desc(c_addr + kb * CROWS * 128 + ks * 32);
+                umma(d, a, b, idesc2, (kb | ks) != 0);
+              }
+          }
+          umma_commit(&empty[st]);
+          umma_commit(&acc_full[buf]);
+        }
+        if (!ok) break;
+        umma_commit(&c_empty[cb]);
+      }
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, abort_flag, p.status, false);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int row = q * 32 + lane;          // TMEM lane = D row
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    const int copy = dup ? (row >> 6) : 0;  // warp-uniform
+    const int col_lo = dup ? copy * 64 : 0, ncols = dup ? 64 : kTileKeys;
+    const float alpha = p.alpha;
+    uint32_t acc_it = 0, epi_ph = 0;
+    int si = 0;
+    bool ok = true;
+    for (int s = blockIdx.x; s < p.n_segs && ok; s += gridDim.x, ++si) {
+      const SegGeom g = seg_geom(p, s);
+      float *lse_buf = lse2 + (si & 1) * 256;
+      // pass 1: per-beacon online log2-sum-exp2 over all keys
+      float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
+      for (int t = 0; t < g.n1; ++t, ++acc_it) {
+        const int buf = acc_it & 1;
+        ok = warp_wait(&acc_full[buf], (acc_it >> 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        tmem_fence_after();
+        const int nvalid = min(kTileKeys, g.L - t * kTileKeys);
+        for (int half = 0; half * 128 < B; ++half) {
+          const int b = half * 128 + (dup ? (row & 63) : row);
+          const bool mine = b < B;
+          float &m = half ? m1 : m0;
+          float &sum = half ? s1 : s0;
+          for (int c0 = col_lo; c0 < col_lo + ncols; c0 += 64) {
+            float v[64];
+            tmem_ld64(tmem_base + lane_addr + buf * 256 + half * 128 + c0, v);
+            const int nv = min(64, nvalid - c0);
+            if (!mine || nv <= 0) continue;
+            float mx[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (i < nv) mx[i & 7] = fmaxf(mx[i & 7], v[i]);
+            const float cm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * alpha;
+            if (cm > m) {
+              sum *= exp2f(m - cm);
+              m = cm;
+            }
+            float ps[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ps[i] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (i < nv) ps[i & 7] += exp2f(fmaf(v[i], alpha, -m));
+            sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+          }
+        }
+        tmem_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      }
+      if (!ok) break;
+      if (dup) {
+        // merge the two copies' partial (max, sum) of each beacon
+        if (copy == 1 && (row & 63) < B) {
+          part[row & 63] = m0;
+          part[64 + (row & 63)] = s0;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi_bar);
+        ok = warp_wait(epi_bar, epi_ph & 1, abort_flag, p.status);
+        ++epi_ph;
+        if (!ok) break;
+        if (copy == 0 && row < B) {
+          const float pm = part[row], psum = part[64 + row];
+          const float mm = fmaxf(m0, pm);
+          s0 = s0 * exp2f(m0 - mm) + psum * exp2f(pm - mm);
+          m0 = mm;
+        }
+      }
+      for (int half = 0; half * 128 < B; ++half) {
+        const int b = half * 128 + row;
+        if (b < B && copy == 0) {
+          const float l2 = (half ? m1 : m0) + log2f(half ? s1 : s0);
+          lse_buf[b] = l2;
+          if (p.lse_out) p.lse_out[g.seg_flat * B + b] = l2 * 0.69314718055994531f;
+          if (l2 != l2) atomicCAS(p.status, kDevOk, kDevNaN);
+        }
+      }
+      // every beacon's lse is in shared memory before any thread reads it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_bar);
+      ok = warp_wait(epi_bar, epi_ph & 1, abort_flag, p.status);
+      ++epi_ph;
+      if (!ok) break;
+      // pass 2: per-key max over beacons of u - lse2
+      for (int t = 0; t < g.n2; ++t, ++acc_it) {
+        const int buf = acc_it & 1;
+        ok = warp_wait(&acc_full[buf], (acc_it >> 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        tmem_fence_after();
+        float bm[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bm[i] = -INFINITY;
+        for (int c0 = 0; c0 < B; c0 += 64) {
+          float v[64];
+          tmem_ld64(tmem_base + lane_addr + buf * 256 + c0, v);
+          const float4 *l4 = reinterpret_cast<const float4 *>(lse_buf + c0);
+#pragma unroll
+          for (int i4 = 0; i4 < 16; ++i4) {
+            if (4 * i4 < B - c0) {
+              const float4 L4 = l4[i4];
+              bm[(4 * i4) & 7] = fmaxf(bm[(4 * i4) & 7], fmaf(v[4 * i4], alpha, -L4.x));
+              bm[(4 * i4 + 1) & 7] = fmaxf(bm[(4 * i4 + 1) & 7], fmaf(v[4 * i4 + 1], alpha, -L4.y));
+              bm[(4 * i4 + 2) & 7] = fmaxf(bm[(4 * i4 + 2) & 7], fmaf(v[4 * i4 + 2], alpha, -L4.z));
+              bm[(4 * i4 + 3) & 7] = fmaxf(bm[(4 * i4 + 3) & 7], fmaf(v[4 * i4 + 3], alpha, -L4.w));
+            }
+          }
+        }
+        tmem_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        const int j = (g.t2 + t) * kTileKeys + row;
+        if (j >= g.P && j < g.L) {
+          const float best = fmaxf(fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3])),
+                                   fmaxf(fmaxf(bm[4], bm[5]), fmaxf(bm[6], bm[7])));
+          const float sc = exp2f(best);
+          if (sc != sc) atomicCAS(p.status, kDevOk, kDevNaN);
+          p.scores[g.seg_flat * p.max_seq + (j - g.P)] = sc;
+        }
+      }
+    }
+  }
+  tmem_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tmem_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// rows x 128 bf16, row stride 256 B, box (64 columns, box_rows rows), 128-byte swizzle
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int CROWS, int NCB>
+cudaError_t launch(const CUtensorMap &km, const CUtensorMap &cm, const TcParams &tp, cudaStream_t s) {
+  const size_t smem = 1024 + (size_t)NCB * CROWS * 256 + (size_t)kStages * kTileKeys * 256 + 256 +
+                      2 * 256 * 4 + 2 * 64 * 4;
+  cudaError_t e = cudaFuncSetAttribute(beacon_score_tc_kernel<CROWS, NCB>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = tp.n_segs < sms ? tp.n_segs : sms;
+  beacon_score_tc_kernel<CROWS, NCB><<<grid, kThreads, smem, s>>>(km, cm, tp);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool beacon_score_tc_supported(int d, int B, int dtype) {
+  return dtype == KVC_BF16 && d == 128 && B >= 32 && B <= 256 && B % 32 == 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_beacon_score_tc(const BeaconScoreParams &p, int n_req, int max_l, cudaStream_t s) {
   (void)max_l;
-  (void)s;
-  return cudaErrorNotSupported;
+  if (!beacon_score_tc_supported(p.d, p.B, p.dtype)) return cudaErrorNotSupported;
+  if (n_req <= 0) return cudaSuccess;
+  CUtensorMap km, cm;
+  const uint64_t krows = (uint64_t)p.layers * (uint64_t)p.num_pages * (uint64_t)p.hkv * kPage;
+  // the beacon map spans every (request, layer, head) segment's B rows
+  const uint64_t crows = (uint64_t)p.total_segs * (uint64_t)p.B;
+  if (krows >= (1ull << 31) || crows >= (1ull << 31)) return cudaErrorInvalidValue;
+  if (!make_map(&km, p.k_pool, krows, kPage) || !make_map(&cm, p.beacons_s, crows, (uint32_t)p.B))
+    return cudaErrorInvalidValue;
+  TcParams tp{};
+  tp.block_table = p.block_table;
+  tp.segs = p.segs;
+  tp.scores = p.scores;
+  tp.lse_out = p.lse_out;
+  tp.status = p.status;
+  tp.num_pages = p.num_pages;
+  tp.bt_stride = p.bt_stride;
+  tp.layers = p.layers;
+  tp.hkv = p.hkv;
+  tp.B = p.B;
+  tp.max_seq = p.max_seq;
+  tp.n_segs = n_req * p.layers * p.hkv;
+  tp.alpha = 1.4426950408889634f / sqrtf(128.0f);
+  if (p.B <= 128) return launch<128, 2>(km, cm, tp, s);
+  return launch<256, 1>(km, cm, tp, s);
 }
 
 }  // namespace kvc

@@ -5,10 +5,11 @@
 // periodic incremental update; BeaconKV abstract: beacons are compact
 // representatives of global query clusters).  project() is the identity.  One
 // CTA per (request, layer, KV head): the beacons sit in shared memory as
-// fp32, each thread assigns whole points (the point in registers, squared
-// distances accumulated dimension by dimension in order, ties to the lower
-// beacon), then one warp per beacon gathers its points in point order with
-// ballots and applies the running mean (n*c + sum)/(n + m).
+// fp32, each thread assigns whole points (the point in registers, loaded as
+// 16-byte vectors; the squared distance in the expanded form |c|^2 - 2 x.c,
+// which has the same argmin, with four partial dot products; ties to the
+// lower beacon), then one warp per beacon gathers its points in point order
+// with ballots and applies the running mean (n*c + sum)/(n + m).
 //
 // Score (the library's definition; the pages leave the importance rule open):
 // z_bj = c_b.k_j/sqrt(d), lse_b = log sum_j exp(z_bj) over every cached key,
@@ -80,23 +81,66 @@ __global__ void __launch_bounds__(kUpdNT) beacon_update_kernel(BeaconUpdateParam
   }
   __syncthreads();
 
-  // assignment: nearest beacon, squared L2, ties to the lower index
+  // squared norms of the beacons, for the expanded distance |c|^2 - 2 x.c
+  // (|x|^2 is the same for every beacon of a point and does not change the argmin)
+  float *cn = reinterpret_cast<float *>(assign + p.W * p.G);  // [B]
+  for (int b = threadIdx.x; b < p.B; b += kUpdNT) {
+    const float4 *c4 = reinterpret_cast<const float4 *>(cs + b * D);
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < D / 4; ++k) {
+      const float4 c = c4[k];
+      a0 = fmaf(c.x, c.x, a0);
+      a1 = fmaf(c.y, c.y, a1);
+      a2 = fmaf(c.z, c.z, a2);
+      a3 = fmaf(c.w, c.w, a3);
+    }
+    cn[b] = (a0 + a1) + (a2 + a3);
+  }
+  __syncthreads();
+
+  // assignment: nearest beacon (smallest |c|^2 - 2 x.c), ties to the lower index
   for (int pt = tid; pt < n_pts; pt += kUpdNT) {
     float x[D];
     const int64_t pb = point_base(pt);
+    if (DT == KVC_BF16) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p.qring) + pb);
 #pragma unroll
-    for (int k = 0; k < D; ++k) x[k] = load_elem<DT>(p.qring, pb + k);
+      for (int v = 0; v < D / 8; ++v) {
+        const uint4 w = src[v];
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          x[8 * v + 2 * e] = __uint_as_float(u[e] << 16);
+          x[8 * v + 2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
+        }
+      }
+    } else {
+      const float4 *src = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(p.qring) + pb);
+#pragma unroll
+      for (int v = 0; v < D / 4; ++v) {
+        const float4 w = src[v];
+        x[4 * v] = w.x;
+        x[4 * v + 1] = w.y;
+        x[4 * v + 2] = w.z;
+        x[4 * v + 3] = w.w;
+      }
+    }
     float best = __int_as_float(0x7f800000);  // +inf
     int besti = 0;
     bool nan = false;
     for (int b = 0; b < p.B; ++b) {
-      const float *c = cs + b * D;
-      float dist = 0.f;
+      const float4 *c4 = reinterpret_cast<const float4 *>(cs + b * D);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-      for (int k = 0; k < D; ++k) {
-        const float diff = x[k] - c[k];
-        dist = fmaf(diff, diff, dist);
+      for (int k = 0; k < D / 4; ++k) {
+        const float4 c = c4[k];
+        a0 = fmaf(x[4 * k], c.x, a0);
+        a1 = fmaf(x[4 * k + 1], c.y, a1);
+        a2 = fmaf(x[4 * k + 2], c.z, a2);
+        a3 = fmaf(x[4 * k + 3], c.w, a3);
       }
+      const float dist = fmaf(-2.f, (a0 + a1) + (a2 + a3), cn[b]);
       nan |= (dist != dist);
       if (dist < best) {
         best = dist;
@@ -246,7 +290,8 @@ __global__ void __launch_bounds__(kScNT) beacon_score_simt_kernel(BeaconScorePar
 cudaError_t launch_beacon_update(const BeaconUpdateParams &p, int n_req, cudaStream_t s) {
   if (n_req <= 0) return cudaSuccess;
   const unsigned grid = (unsigned)(n_req * p.layers * p.hkv);
-  const size_t smem = (size_t)p.B * p.d * sizeof(float) + (size_t)p.W * p.G * sizeof(int32_t);
+  const size_t smem = (size_t)p.B * p.d * sizeof(float) + (size_t)p.W * p.G * sizeof(int32_t) +
+                      (size_t)p.B * sizeof(float);
   cudaError_t e = cudaErrorInvalidValue;
 #define KVC_UPD(DV, DTV)                                                                      \
   if (p.d == DV && p.dtype == DTV) {                                                          \

@@ -203,7 +203,10 @@ kvc_status take_device_status(kvc_ctx *ctx) {
   if (dev_status == kDevOk) return KVC_OK;
   KVC_CUDA(ctx, cudaMemsetAsync(ctx->d_status, 0, 4, ctx->stream));
   KVC_CUDA(ctx, cudaStreamSynchronize(ctx->stream));
-  return fail(ctx, dev_status == kDevNaN ? KVC_ERR_NAN : KVC_ERR_DEVICE_CHECK,
+  return fail(ctx,
+              dev_status == kDevNaN       ? KVC_ERR_NAN
+              : dev_status == kDevTimeout ? KVC_ERR_DEVICE_TIMEOUT
+                                          : KVC_ERR_DEVICE_CHECK,
               "device reported an error (status word " + std::to_string(dev_status) + ")");
 }
 
@@ -584,6 +587,7 @@ kvc_status kvc_compress(kvc_ctx *ctx, kvc_selector selector, const int32_t *budg
     bp.lse_out = ctx->d_lse;
     bp.status = ctx->d_status;
     bp.num_pages = c.num_pages;
+    bp.total_segs = (int64_t)R * per_req_segs;
     bp.bt_stride = ctx->maxp;
     bp.layers = c.num_layers;
     bp.hkv = c.num_kv_heads;
@@ -599,6 +603,7 @@ kvc_status kvc_compress(kvc_ctx *ctx, kvc_selector selector, const int32_t *budg
                : launch_beacon_score_simt(bp, (int)segs.size(), ctx->stream);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "beacon_score");
     st.launches += 1;
+    st.score_kernel = use_tc ? 2 : 1;
   }
   if (timed) KVC_CUDA(ctx, cudaEventRecord(ctx->ev[1], ctx->stream));
   SelectCompactParams sp{};

@@ -19,6 +19,7 @@ constexpr int kMaxRowBytes = 1024;
 constexpr int kDevOk = 0;
 constexpr int kDevNaN = 1;
 constexpr int kDevIndex = 2;
+constexpr int kDevTimeout = 3;  // a bounded device wait ran out
 
 // Score sources of the fused select + compaction kernel.
 enum ScoreMode : int { kModeRandom = 0, kModeRandomShared = 1, kModeScores = 2 };
@@ -69,6 +70,7 @@ struct BeaconScoreParams {
   float *lse_out;             // optional [R][layers][Hkv][B]
   int32_t *status;
   int64_t num_pages;
+  int64_t total_segs;         // R * layers * Hkv (rows of the beacon arrays / B)
   int32_t bt_stride, layers, hkv, B, d, dtype, max_seq;
 };
 

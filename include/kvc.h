@@ -120,6 +120,8 @@ typedef struct {
   float ms_select_compact;       /* device time of the fused select + compaction kernel */
   float ms_total;                /* device time of the whole call */
   int32_t launches;              /* kernels this call launched */
+  int32_t score_kernel;          /* beacon score kernel used: 0 none, 1 SIMT fp32, 2 tcgen05 */
+  int32_t reserved;
 } kvc_round_stats;
 
 /* Zero-copy view of the context's device state (pointers into the pools and

@@ -157,3 +157,20 @@ def test_long_trace_sampled():
     w = wl.scaled(wl.long_trace(), num_requests=2, num_layers=4)
     out = run_beacon(w, sample=3)
     print(out)
+
+
+@pytest.mark.parametrize("impl", [1, 2], ids=["simt", "tcgen05"])
+def test_score_kernels_small(impl):
+    """Both beacon-score kernels (SIMT fp32 and tcgen05) against the oracle."""
+    out = run_beacon(wl.beacon_serving(R=2, layers=2), score_impl=impl)
+    print(impl, out)
+
+
+def test_tcgen05_256_beacons():
+    """The 256-beacon path of the tensor-core kernel (two M=128 halves in pass 1)."""
+    w = wl.scaled(wl.long_trace(), num_requests=1, num_layers=2)
+    w.length = np.array([4133])
+    w.budget = np.array([1000])
+    w.prompt = np.array([77])
+    out = run_beacon(w, score_impl=2)
+    print(out)
