@@ -25,8 +25,10 @@
 // load per (page, 64-column half): a page holds 16 keys x 256 B contiguous,
 // the tensor map covers the whole pool as rows of 128 bf16, 128-byte
 // swizzle); warp 1 issues the MMAs (one elected lane) and commits them to
-// mbarriers; warps 2-5 run the epilogue (tcgen05.ld of 64 columns at a time;
-// sums and maxima in 8 independent partials to keep the pipes busy).
+// mbarriers; warps 2-9 run the epilogue in two groups of four, group g taking
+// the tiles whose accumulator is in TMEM buffer g (tcgen05.ld of 64 columns
+// at a time; sums and maxima in 8 independent partials; the per-beacon
+// partial (max, sum) of the groups merged once per segment).
 // Key tiles rotate through 4 shared-memory stages; the accumulators through
 // two 256-column TMEM buffers.  No load uses cluster multicast.
 // Every mbarrier wait is bounded (2 s of %globaltimer): on expiry the kernel
@@ -42,7 +44,8 @@ namespace {
 
 constexpr int kTileKeys = 128;
 constexpr int kStages = 4;
-constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kEpiWarps = 8;   // two groups of 4: group g drains accumulator buffer g
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(epi_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *lse2 = reinterpret_cast<float *>(tmem_slot + 4);  // [2][256]
-  float *part = lse2 + 512;                                 // [2][64] (m, sum) of the upper copy
+  float *part = lse2 + 512;                                 // [4][2][256] partial (m, sum)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&c_empty[i], 1);
     }
     mbar_init(mma_done, 1);
-    mbar_init(epi_bar, 4);
+    mbar_init(epi_bar, kEpiWarps);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -340,11 +343,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
+    // Group grp (warps 2-5 or 6-9) handles the tiles whose accumulator sits
+    // in buffer grp, i.e. every other tile; each warp reads the TMEM lane
+    // quarter (warp % 4) it may access.
+    const int ew = warp - 2, grp = ew >> 2;
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int row = q * 32 + lane;          // TMEM lane = D row
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     const int copy = dup ? (row >> 6) : 0;  // warp-uniform
     const int col_lo = dup ? copy * 64 : 0, ncols = dup ? 64 : kTileKeys;
+    const int nslot = dup ? 4 : 2;          // partials per beacon: groups x copies
+    const int slot = grp * (dup ? 2 : 1) + copy;
     const float alpha = p.alpha;
     uint32_t acc_it = 0, epi_ph = 0;
     int si = 0;
@@ -352,10 +361,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = blockIdx.x; s < p.n_segs && ok; s += gridDim.x, ++si) {
       const SegGeom g = seg_geom(p, s);
       float *lse_buf = lse2 + (si & 1) * 256;
-      // pass 1: per-beacon online log2-sum-exp2 over all keys
+      // pass 1: per-beacon online log2-sum-exp2 over this group's tiles
       float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
       for (int t = 0; t < g.n1; ++t, ++acc_it) {
         const int buf = acc_it & 1;
+        if (buf != grp) continue;
         ok = warp_wait(&acc_full[buf], (acc_it >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
         tmem_fence_after();
@@ -396,31 +406,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
       }
       if (!ok) break;
-      if (dup) {
-        // merge the two copies' partial (max, sum) of each beacon
-        if (copy == 1 && (row & 63) < B) {
-          part[row & 63] = m0;
-          part[64 + (row & 63)] = s0;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(epi_bar);
-        ok = warp_wait(epi_bar, epi_ph & 1, abort_flag, p.status);
-        ++epi_ph;
-        if (!ok) break;
-        if (copy == 0 && row < B) {
-          const float pm = part[row], psum = part[64 + row];
-          const float mm = fmaxf(m0, pm);
-          s0 = s0 * exp2f(m0 - mm) + psum * exp2f(pm - mm);
-          m0 = mm;
+      // merge the partial (max, sum) of each beacon over groups and copies
+      for (int half = 0; half * 128 < B; ++half) {
+        const int b = half * 128 + (dup ? (row & 63) : row);
+        if (b < B) {
+          part[(slot * 2 + 0) * 256 + b] = half ? m1 : m0;
+          part[(slot * 2 + 1) * 256 + b] = half ? s1 : s0;
         }
       }
-      for (int half = 0; half * 128 < B; ++half) {
-        const int b = half * 128 + row;
-        if (b < B && copy == 0) {
-          const float l2 = (half ? m1 : m0) + log2f(half ? s1 : s0);
-          lse_buf[b] = l2;
-          if (p.lse_out) p.lse_out[g.seg_flat * B + b] = l2 * 0.69314718055994531f;
-          if (l2 != l2) atomicCAS(p.status, kDevOk, kDevNaN);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_bar);
+      ok = warp_wait(epi_bar, epi_ph & 1, abort_flag, p.status);
+      ++epi_ph;
+      if (!ok) break;
+      if (slot == 0) {
+        for (int half = 0; half * 128 < B; ++half) {
+          const int b = half * 128 + row;
+          if (b < B) {
+            float mm = -INFINITY;
+            for (int k = 0; k < nslot; ++k) mm = fmaxf(mm, part[(k * 2) * 256 + b]);
+            float ss = 0.f;
+            for (int k = 0; k < nslot; ++k) {
+              const float pm = part[(k * 2) * 256 + b];
+              if (pm != -INFINITY) ss += part[(k * 2 + 1) * 256 + b] * exp2f(pm - mm);
+            }
+            const float l2 = mm + log2f(ss);
+            lse_buf[b] = l2;
+            if (p.lse_out) p.lse_out[g.seg_flat * B + b] = l2 * 0.69314718055994531f;
+            if (l2 != l2) atomicCAS(p.status, kDevOk, kDevNaN);
+          }
         }
       }
       // every beacon's lse is in shared memory before any thread reads it
@@ -429,9 +443,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = warp_wait(epi_bar, epi_ph & 1, abort_flag, p.status);
       ++epi_ph;
       if (!ok) break;
-      // pass 2: per-key max over beacons of u - lse2
+      // pass 2: per-key max over beacons of u - lse2 (this group's tiles)
       for (int t = 0; t < g.n2; ++t, ++acc_it) {
         const int buf = acc_it & 1;
+        if (buf != grp) continue;
         ok = warp_wait(&acc_full[buf], (acc_it >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
         tmem_fence_after();
@@ -444,13 +459,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float4 *l4 = reinterpret_cast<const float4 *>(lse_buf + c0);
 #pragma unroll
           for (int i4 = 0; i4 < 16; ++i4) {
-            if (4 * i4 < B - c0) {
-              const float4 L4 = l4[i4];
-              bm[(4 * i4) & 7] = fmaxf(bm[(4 * i4) & 7], fmaf(v[4 * i4], alpha, -L4.x));
-              bm[(4 * i4 + 1) & 7] = fmaxf(bm[(4 * i4 + 1) & 7], fmaf(v[4 * i4 + 1], alpha, -L4.y));
-              bm[(4 * i4 + 2) & 7] = fmaxf(bm[(4 * i4 + 2) & 7], fmaf(v[4 * i4 + 2], alpha, -L4.z));
-              bm[(4 * i4 + 3) & 7] = fmaxf(bm[(4 * i4 + 3) & 7], fmaf(v[4 * i4 + 3], alpha, -L4.w));
-            }
+            const float4 L4 = l4[i4];
+            bm[(4 * i4) & 7] = fmaxf(bm[(4 * i4) & 7], fmaf(v[4 * i4], alpha, -L4.x));
+            bm[(4 * i4 + 1) & 7] = fmaxf(bm[(4 * i4 + 1) & 7], fmaf(v[4 * i4 + 1], alpha, -L4.y));
+            bm[(4 * i4 + 2) & 7] = fmaxf(bm[(4 * i4 + 2) & 7], fmaf(v[4 * i4 + 2], alpha, -L4.z));
+            bm[(4 * i4 + 3) & 7] = fmaxf(bm[(4 * i4 + 3) & 7], fmaf(v[4 * i4 + 3], alpha, -L4.w));
           }
         }
         tmem_fence_before();
@@ -503,7 +516,7 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows
 template <int CROWS, int NCB>
 cudaError_t launch(const CUtensorMap &km, const CUtensorMap &cm, const TcParams &tp, cudaStream_t s) {
   const size_t smem = 1024 + (size_t)NCB * CROWS * 256 + (size_t)kStages * kTileKeys * 256 + 256 +
-                      2 * 256 * 4 + 2 * 64 * 4;
+                      2 * 256 * 4 + 4 * 2 * 256 * 4;
   cudaError_t e = cudaFuncSetAttribute(beacon_score_tc_kernel<CROWS, NCB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -518,7 +531,7 @@ cudaError_t launch(const CUtensorMap &km, const CUtensorMap &cm, const TcParams 
 }  // namespace
 
 bool beacon_score_tc_supported(int d, int B, int dtype) {
-  return dtype == KVC_BF16 && d == 128 && B >= 32 && B <= 256 && B % 32 == 0 && encode_fn() != nullptr;
+  return dtype == KVC_BF16 && d == 128 && B >= 64 && B <= 256 && B % 64 == 0 && encode_fn() != nullptr;
 }
 
 cudaError_t launch_beacon_score_tc(const BeaconScoreParams &p, int n_req, int max_l, cudaStream_t s) {
