@@ -47,6 +47,7 @@ KVC_SEL_RANDOM_SHARED = 1
 KVC_SEL_BEACON = 2
 
 KVC_OPT_BEACON_SCORE_IMPL = 0
+KVC_OPT_BEACON_UPDATE_IMPL = 1
 
 SELECTORS = {"random": KVC_SEL_RANDOM, "random_shared": KVC_SEL_RANDOM_SHARED,
              "beacon": KVC_SEL_BEACON}

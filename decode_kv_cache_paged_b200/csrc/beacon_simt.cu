@@ -5,11 +5,12 @@
 // periodic incremental update; BeaconKV abstract: beacons are compact
 // representatives of global query clusters).  project() is the identity.  One
 // CTA per (request, layer, KV head): the beacons sit in shared memory as
-// fp32, each thread assigns whole points (the point in registers, loaded as
-// 16-byte vectors; the squared distance in the expanded form |c|^2 - 2 x.c,
-// which has the same argmin, with four partial dot products; ties to the
-// lower beacon), then one warp per beacon gathers its points in point order
-// with ballots and applies the running mean (n*c + sum)/(n + m).
+// fp32; the points are assigned in blocks of 64 with a register-tiled
+// product (each thread 4 points x B/16 beacons, float4 operands, 8 FMAs per
+// shared-memory load) on the expanded distance |c|^2 - 2 x.c, which has the
+// same argmin; ties go to the lower beacon.  Then one warp per beacon gathers
+// its points in point order with ballots and applies the running mean
+// (n*c + sum)/(n + m).
 //
 // Score (the library's definition; the pages leave the importance rule open):
 // z_bj = c_b.k_j/sqrt(d), lse_b = log sum_j exp(z_bj) over every cached key,
@@ -47,12 +48,19 @@ __device__ __forceinline__ void set_status(int32_t *status, int code) {
 }
 
 constexpr int kUpdNT = 256;
+constexpr int kPB = 64;  // points per assignment block
 
+// One (request, layer, KV head) segment per CTA.  Shared memory: the beacons
+// as fp32 rows padded to D+4 floats, a block of kPB points likewise, the
+// beacons' squared norms and the assignment of every point.
 template <int D, int DT>
 __global__ void __launch_bounds__(kUpdNT) beacon_update_kernel(BeaconUpdateParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
-  float *cs = reinterpret_cast<float *>(smem);                 // [B][D]
-  int32_t *assign = reinterpret_cast<int32_t *>(cs + p.B * D);  // [n_pts]
+  constexpr int RS = D + 4;  // padded row stride (floats)
+  float *cs = reinterpret_cast<float *>(smem);  // [B][RS]
+  float *xs = cs + p.B * RS;                     // [kPB][RS]
+  float *cn = xs + kPB * RS;                     // [B]
+  int32_t *assign = reinterpret_cast<int32_t *>(cn + p.B);  // [W*G]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x % p.hkv;
   const int l = (blockIdx.x / p.hkv) % p.layers;
@@ -74,83 +82,115 @@ __global__ void __launch_bounds__(kUpdNT) beacon_update_kernel(BeaconUpdateParam
     const int b = e / D, k = e - b * D;
     if (ud.init) {
       const int src = (int)(((int64_t)b * n_pts) / p.B);
-      cs[e] = load_elem<DT>(p.qring, point_base(src) + k);
+      cs[b * RS + k] = load_elem<DT>(p.qring, point_base(src) + k);
     } else {
-      cs[e] = gbeac[e];
+      cs[b * RS + k] = gbeac[e];
     }
   }
   __syncthreads();
-
   // squared norms of the beacons, for the expanded distance |c|^2 - 2 x.c
-  // (|x|^2 is the same for every beacon of a point and does not change the argmin)
-  float *cn = reinterpret_cast<float *>(assign + p.W * p.G);  // [B]
-  for (int b = threadIdx.x; b < p.B; b += kUpdNT) {
-    const float4 *c4 = reinterpret_cast<const float4 *>(cs + b * D);
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < D / 4; ++k) {
-      const float4 c = c4[k];
-      a0 = fmaf(c.x, c.x, a0);
-      a1 = fmaf(c.y, c.y, a1);
-      a2 = fmaf(c.z, c.z, a2);
-      a3 = fmaf(c.w, c.w, a3);
-    }
-    cn[b] = (a0 + a1) + (a2 + a3);
+  // (|x|^2 is the same for every beacon of a point and does not move the argmin)
+  for (int b = tid; b < p.B; b += kUpdNT) {
+    float a = 0.f;
+    for (int k = 0; k < D; ++k) a = fmaf(cs[b * RS + k], cs[b * RS + k], a);
+    cn[b] = a;
   }
-  __syncthreads();
 
-  // assignment: nearest beacon (smallest |c|^2 - 2 x.c), ties to the lower index
-  for (int pt = tid; pt < n_pts; pt += kUpdNT) {
-    float x[D];
-    const int64_t pb = point_base(pt);
-    if (DT == KVC_BF16) {
-      const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p.qring) + pb);
-#pragma unroll
-      for (int v = 0; v < D / 8; ++v) {
-        const uint4 w = src[v];
-        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[8 * v + 2 * e] = __uint_as_float(u[e] << 16);
-          x[8 * v + 2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
+  // assignment, kPB points at a time: thread (ty, tx) owns points 4ty..4ty+3
+  // of the block and beacons tx, tx+16, ...; dot products accumulate in k order
+  constexpr int kMaxNB = kMaxBeacons / 16;
+  const int ty = tid >> 4, tx = tid & 15;
+  const int NB = (p.B + 15) >> 4;  // beacons tx + 16 j, j < NB, that are < B
+  bool nan = false;
+  for (int p0 = 0; p0 < n_pts; p0 += kPB) {
+    __syncthreads();  // xs reuse
+    constexpr int kVec = (DT == KVC_BF16) ? 8 : 4;  // elements per 16-byte load
+    constexpr int kChunks = D / kVec;
+    for (int e = tid; e < kPB * kChunks; e += kUpdNT) {
+      const int pi = e / kChunks, c = e - pi * kChunks;
+      const int pt = p0 + pi;
+      float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+      if (pt < n_pts) {
+        const uint8_t *src = p.qring + (point_base(pt) + c * kVec) * (DT == KVC_BF16 ? 2 : 4);
+        const uint4 w = *reinterpret_cast<const uint4 *>(src);
+        if (DT == KVC_BF16) {
+          lo = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                           __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+          hi = make_float4(__uint_as_float(w.z << 16), __uint_as_float(w.z & 0xffff0000u),
+                           __uint_as_float(w.w << 16), __uint_as_float(w.w & 0xffff0000u));
+        } else {
+          lo = make_float4(__uint_as_float(w.x), __uint_as_float(w.y), __uint_as_float(w.z),
+                           __uint_as_float(w.w));
         }
       }
-    } else {
-      const float4 *src = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(p.qring) + pb);
+      float4 *dst = reinterpret_cast<float4 *>(xs + pi * RS + c * kVec);
+      dst[0] = lo;
+      if (DT == KVC_BF16) dst[1] = hi;
+    }
+    __syncthreads();
+    float acc[4][kMaxNB];
 #pragma unroll
-      for (int v = 0; v < D / 4; ++v) {
-        const float4 w = src[v];
-        x[4 * v] = w.x;
-        x[4 * v + 1] = w.y;
-        x[4 * v + 2] = w.z;
-        x[4 * v + 3] = w.w;
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < kMaxNB; ++j) acc[i][j] = 0.f;
+    const float4 *x4 = reinterpret_cast<const float4 *>(xs) + (ty * 4) * (RS / 4);
+    const float4 *c4 = reinterpret_cast<const float4 *>(cs) + tx * (RS / 4);
+#pragma unroll 2
+    for (int k4 = 0; k4 < D / 4; ++k4) {
+      float4 xv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[i] = x4[i * (RS / 4) + k4];
+#pragma unroll
+      for (int j = 0; j < kMaxNB; ++j) {
+        if (j < NB) {
+          const float4 cv = c4[j * 16 * (RS / 4) + k4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float a = acc[i][j];
+            a = fmaf(xv[i].x, cv.x, a);
+            a = fmaf(xv[i].y, cv.y, a);
+            a = fmaf(xv[i].z, cv.z, a);
+            a = fmaf(xv[i].w, cv.w, a);
+            acc[i][j] = a;
+          }
+        }
       }
     }
-    float best = __int_as_float(0x7f800000);  // +inf
-    int besti = 0;
-    bool nan = false;
-    for (int b = 0; b < p.B; ++b) {
-      const float4 *c4 = reinterpret_cast<const float4 *>(cs + b * D);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    // argmin over this thread's beacons, then over the 16 threads of the row
 #pragma unroll
-      for (int k = 0; k < D / 4; ++k) {
-        const float4 c = c4[k];
-        a0 = fmaf(x[4 * k], c.x, a0);
-        a1 = fmaf(x[4 * k + 1], c.y, a1);
-        a2 = fmaf(x[4 * k + 2], c.z, a2);
-        a3 = fmaf(x[4 * k + 3], c.w, a3);
+    for (int i = 0; i < 4; ++i) {
+      float best = __int_as_float(0x7f800000);
+      int besti = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < kMaxNB; ++j) {
+        const int b = tx + 16 * j;
+        if (j < NB && b < p.B) {
+          const float dist = fmaf(-2.f, acc[i][j], cn[b]);
+          nan |= (dist != dist);
+          if (dist < best) {
+            best = dist;
+            besti = b;
+          }
+        }
       }
-      const float dist = fmaf(-2.f, (a0 + a1) + (a2 + a3), cn[b]);
-      nan |= (dist != dist);
-      if (dist < best) {
-        best = dist;
-        besti = b;
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, besti, o);
+        if (ob < best || (ob == best && oi < besti)) {
+          best = ob;
+          besti = oi;
+        }
+      }
+      const int pt = p0 + ty * 4 + i;
+      if (tx == 0 && pt < n_pts) {
+        const int a = besti == 0x7fffffff ? 0 : besti;  // all distances NaN: flagged below
+        assign[pt] = a;
+        if (p.assign_out) p.assign_out[seg * (int64_t)(p.W * p.G) + pt] = a;
       }
     }
-    if (nan) set_status(p.status, kDevNaN);
-    assign[pt] = besti;
-    if (p.assign_out) p.assign_out[seg * (int64_t)(p.W * p.G) + pt] = besti;
   }
+  if (nan) set_status(p.status, kDevNaN);
   __syncthreads();
 
   // running mean, one warp per beacon, points in order
@@ -176,7 +216,7 @@ __global__ void __launch_bounds__(kUpdNT) beacon_update_kernel(BeaconUpdateParam
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
       const int e = b * D + lane + 32 * k;
-      float v = cs[e];
+      float v = cs[b * RS + lane + 32 * k];
       if (m > 0) v = ((float)n * v + sum[k]) / (float)(n + m);
       gbeac[e] = v;
       store_scoring<DT>(p.beacons_s, seg * p.B * D + e, v);
@@ -290,8 +330,8 @@ __global__ void __launch_bounds__(kScNT) beacon_score_simt_kernel(BeaconScorePar
 cudaError_t launch_beacon_update(const BeaconUpdateParams &p, int n_req, cudaStream_t s) {
   if (n_req <= 0) return cudaSuccess;
   const unsigned grid = (unsigned)(n_req * p.layers * p.hkv);
-  const size_t smem = (size_t)p.B * p.d * sizeof(float) + (size_t)p.W * p.G * sizeof(int32_t) +
-                      (size_t)p.B * sizeof(float);
+  const size_t smem = sizeof(float) * ((size_t)p.B * (p.d + 4) + (size_t)kPB * (p.d + 4) + p.B) +
+                      (size_t)p.W * p.G * sizeof(int32_t);
   cudaError_t e = cudaErrorInvalidValue;
 #define KVC_UPD(DV, DTV)                                                                      \
   if (p.d == DV && p.dtype == DTV) {                                                          \

@@ -1,0 +1,282 @@
+// beacon_update_tc.cu -- BeaconKV periodic beacon update with the nearest-
+// beacon assignment on the tensor cores (bf16 query ring, head_dim 128).
+//
+// What it computes (BeaconKV explainer §3.2: a query goes to its nearest
+// beacon; beacons are updated periodically and incrementally): every point
+// (a query of one of the G query heads of the KV head, over the steps since
+// the previous update) is assigned to the beacon with the smallest squared
+// distance, ties to the lower index, against the beacons as they were before
+// this update; each beacon with m new points becomes (n c + sum)/(n + m).
+//
+// Assignment as a product: |x - c|^2 = |x|^2 + |c|^2 - 2 x.c and |x|^2 does
+// not depend on the beacon, so the argmin is that of |c|^2 - 2 x.c.  The
+// points are bf16 (exact as MMA operands); the fp32 beacons enter as two bf16
+// terms, c = c_hi + c_lo + r with |r_k| <= 2^-18 |c_k|, so x.c is computed
+// as x.c_hi + x.c_lo with one fp32 accumulation in TMEM and an error of at
+// most 2^-18 sum_k |x_k c_k| beyond fp32 rounding.  |c|^2 is the fp32 norm of
+// the fp32 beacon.  One CTA of 128 threads per (request, layer, KV head):
+// tiles of 128 points (TMEM lane = point) against all B beacons (N = B).
+// Then a stable counting sort of the points by beacon (warp match) and one
+// warp per beacon summing its points in point order.
+#include <cuda_bf16.h>
+
+#include "kvc_internal.h"
+#include "tc_ptx.cuh"
+
+namespace kvc {
+namespace {
+
+constexpr int kUT = 128;  // threads: one point of the 128-point tile each
+
+// Byte offset of bf16 element k (0..63) of `row` inside one 64-element
+// K-block of a K-major tile in the 128-byte-swizzled canonical layout.
+__device__ __forceinline__ uint32_t sw128_off(int row, int k) {
+  return (uint32_t)row * 128u + ((uint32_t)((k >> 3) ^ (row & 7)) << 4) + (uint32_t)(k & 7) * 2u;
+}
+
+__global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParams p, uint32_t tmem_cols) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int D = 128;
+  const int B = p.B, NP = p.W * p.G;
+  uint8_t *xs = smem;                    // [2 K-blocks][128 rows][128 B]
+  uint8_t *chi = xs + 32768;             // [2][B][128 B]
+  uint8_t *clo = chi + B * 256;          // [2][B][128 B]
+  float *cn = reinterpret_cast<float *>(clo + B * 256);  // [B]
+  float *cpart = cn + B;                                  // [4][B]
+  int32_t *assign = reinterpret_cast<int32_t *>(cpart + 4 * B);  // [NP]
+  int32_t *order = assign + NP;                                   // [NP]
+  int32_t *offs = order + NP;                                     // [B + 1]
+  int32_t *cursor = offs + B + 1;                                 // [B]
+  uint64_t *mbar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(cursor + B) + 15) & ~uintptr_t(15));
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.x % p.hkv;
+  const int l = (blockIdx.x / p.hkv) % p.layers;
+  const UpdateDesc ud = p.descs[blockIdx.x / (p.hkv * p.layers)];
+  const int r = ud.req;
+  const int n_pts = ud.n_steps * p.G;
+  const int64_t seg = ((int64_t)r * p.layers + l) * p.hkv + h;
+  float *gbeac = p.beacons + seg * B * D;
+  int32_t *gcnt = p.counts + seg * B;
+  const __nv_bfloat16 *ring = reinterpret_cast<const __nv_bfloat16 *>(p.qring);
+  auto point_base = [&](int pt) -> int64_t {
+    const int step = pt / p.G, g = pt - step * p.G;
+    const int slot = (ud.ring_start + step) % p.W;
+    return ((((int64_t)r * p.layers + l) * p.W + slot) * p.hq + (h * p.G + g)) * D;
+  };
+  // beacon b's value before this update, element k (first update: a point)
+  auto c_old = [&](int b, int k) -> float {
+    if (ud.init) return __bfloat162float(ring[point_base((int)(((int64_t)b * n_pts) / B)) + k]);
+    return gbeac[b * D + k];
+  };
+
+  if (tid == 0) {
+    mbar_init(mbar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                 "r"(tmem_cols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+
+  // beacons: bf16 hi/lo terms in the swizzled layout, fp32 squared norms
+  for (int b0 = 0; b0 < B; b0 += 4) {  // B is a multiple of 32
+    float c[4], sq[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) c[u] = c_old(b0 + u, tid);
+    const int kb = tid >> 6, k = tid & 63;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(c[u]);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(c[u] - __bfloat162float(hi));
+      *reinterpret_cast<__nv_bfloat16 *>(chi + kb * B * 128 + sw128_off(b0 + u, k)) = hi;
+      *reinterpret_cast<__nv_bfloat16 *>(clo + kb * B * 128 + sw128_off(b0 + u, k)) = lo;
+      sq[u] = c[u] * c[u];
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) sq[u] += __shfl_xor_sync(0xffffffffu, sq[u], o);
+    if (lane == 0)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) cpart[warp * B + b0 + u] = sq[u];
+  }
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t tmem_base = *tslot;
+  for (int b = tid; b < B; b += kUT) cn[b] = ((cpart[b] + cpart[B + b]) + cpart[2 * B + b]) + cpart[3 * B + b];
+
+  // assignment, 128 points per tile
+  const uint32_t idesc = idesc_bf16_f32(128, B);
+  const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+  bool nan = false;
+  int tile = 0;
+  for (int p0 = 0; p0 < n_pts; p0 += 128, ++tile) {
+    const int pt = p0 + tid;
+    if (pt < n_pts) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(ring + point_base(pt));
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 w = src[c];
+        *reinterpret_cast<uint4 *>(xs + (c >> 3) * 16384 + tid * 128 + (((c & 7) ^ (tid & 7)) << 4)) = w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        *reinterpret_cast<uint4 *>(xs + (c >> 3) * 16384 + tid * 128 + (((c & 7) ^ (tid & 7)) << 4)) =
+            make_uint4(0, 0, 0, 0);
+    }
+    // the tensor core reads shared memory through the async proxy
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tmem_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tmem_fence_after();
+      const uint32_t xa = smem_u32(xs), ha = smem_u32(chi), la = smem_u32(clo);
+      for (int term = 0; term < 2; ++term)
+        for (int kb = 0; kb < 2; ++kb)
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t a = sw128_desc(xa + kb * 16384 + ks * 32);
+            const uint64_t bd = sw128_desc((term ? la : ha) + kb * B * 128 + ks * 32);
+            umma(tmem_base, a, bd, idesc, (term | kb | ks) != 0);
+          }
+      umma_commit(mbar);
+      if (!mbar_wait(mbar, tile & 1, abort_flag, p.status)) *abort_flag = 1;
+    }
+    __syncthreads();
+    if (*abort_flag) break;
+    tmem_fence_after();
+    float best = __int_as_float(0x7f800000);
+    int besti = 0;
+    for (int c0 = 0; c0 < B; c0 += 32) {
+      float v[32];
+      tmem_ld32(tmem_base + lane_addr + c0, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float dist = fmaf(-2.f, v[i], cn[c0 + i]);
+        nan |= (dist != dist);
+        if (dist < best) {
+          best = dist;
+          besti = c0 + i;
+        }
+      }
+    }
+    if (pt < n_pts) {
+      assign[pt] = besti;
+      if (p.assign_out) p.assign_out[seg * (int64_t)NP + pt] = besti;
+    }
+    tmem_fence_before();
+    __syncthreads();  // xs and the accumulator are rewritten by the next tile
+  }
+  if (nan) atomicCAS(p.status, kDevOk, kDevNaN);
+
+  if (!*abort_flag) {
+    // stable counting sort of the points by beacon
+    for (int b = tid; b <= B; b += kUT) offs[b] = 0;
+    __syncthreads();
+    for (int pt = tid; pt < n_pts; pt += kUT) atomicAdd(&offs[assign[pt] + 1], 1);
+    __syncthreads();
+    if (warp == 0) {
+      int carry = 0;
+      for (int b0 = 0; b0 <= B; b0 += 32) {
+        const int b = b0 + lane;
+        int v = b <= B ? offs[b] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += u;
+        }
+        if (b <= B) offs[b] = v + carry;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+      __syncwarp();
+      for (int b = lane; b < B; b += 32) cursor[b] = offs[b];
+      __syncwarp();
+      for (int c0 = 0; c0 < n_pts; c0 += 32) {
+        const int pt = c0 + lane;
+        const int a = pt < n_pts ? assign[pt] : -1 - lane;  // distinct for lanes past the end
+        const unsigned peers = __match_any_sync(0xffffffffu, a);
+        const int leader = __ffs(peers) - 1;
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        int base = (lane == leader && a >= 0) ? cursor[a] : 0;
+        base = __shfl_sync(0xffffffffu, base, leader);
+        if (a >= 0) order[base + rank] = pt;
+        __syncwarp();
+        if (lane == leader && a >= 0) cursor[a] = base + __popc(peers);
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    // running mean, one warp per beacon, its points in point order
+    for (int b = warp; b < B; b += kUT / 32) {
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      const int o0 = offs[b], m = offs[b + 1] - o0;
+      int i = 0;
+      for (; i + 4 <= m; i += 4) {
+        float x[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t pb = point_base(order[o0 + i + u]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) x[u][j] = __bfloat162float(ring[pb + lane + 32 * j]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) sum[j] += x[u][j];
+      }
+      for (; i < m; ++i) {
+        const int64_t pb = point_base(order[o0 + i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sum[j] += __bfloat162float(ring[pb + lane + 32 * j]);
+      }
+      const int n = ud.init ? 0 : gcnt[b];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int k = lane + 32 * j;
+        float v = c_old(b, k);
+        if (m > 0) v = ((float)n * v + sum[j]) / (float)(n + m);
+        gbeac[b * D + k] = v;
+        reinterpret_cast<__nv_bfloat16 *>(p.beacons_s)[seg * B * D + b * D + k] = __float2bfloat16_rn(v);
+      }
+      if (lane == 0) gcnt[b] = n + m;
+    }
+  }
+  tmem_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tmem_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(tmem_cols));
+  }
+}
+
+}  // namespace
+
+bool beacon_update_tc_supported(int d, int B, int dtype) {
+  return dtype == KVC_BF16 && d == 128 && B >= 32 && B <= 256 && B % 32 == 0;
+}
+
+cudaError_t launch_beacon_update_tc(const BeaconUpdateParams &p, int n_req, cudaStream_t s) {
+  if (!beacon_update_tc_supported(p.d, p.B, p.dtype)) return cudaErrorNotSupported;
+  if (n_req <= 0) return cudaSuccess;
+  const int NP = p.W * p.G;
+  // x tile, c_hi/c_lo tiles, cn + cpart[4] + cursor (6 floats/ints per beacon),
+  // assign + order (2 ints per point), offs (B + 1), barrier/slot/flag
+  const size_t smem = 1024 + 32768 + (size_t)p.B * 512 + (size_t)p.B * 4 * 6 + (size_t)NP * 8 +
+                      (size_t)(p.B + 1) * 4 + 64;
+  uint32_t cols = 32;
+  while ((int)cols < p.B) cols <<= 1;
+  cudaError_t e = cudaFuncSetAttribute(beacon_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  beacon_update_tc_kernel<<<(unsigned)(n_req * p.layers * p.hkv), kUT, smem, s>>>(p, cols);
+  return cudaGetLastError();
+}
+
+}  // namespace kvc

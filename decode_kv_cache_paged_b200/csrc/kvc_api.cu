@@ -118,6 +118,7 @@ struct kvc_ctx {
   std::vector<int32_t> free_pages;
   int64_t round = 0;
   int score_impl = 0;
+  int update_impl = 0;
   int es = 2, row_bytes = 0, G = 1, maxp = 0;
   std::string err;
 };
@@ -357,6 +358,12 @@ kvc_status kvc_set_option(kvc_ctx *ctx, kvc_option opt, int64_t value) {
         return fail(ctx, KVC_ERR_UNSUPPORTED, "tcgen05 beacon score not available for this config");
       ctx->score_impl = (int)value;
       return KVC_OK;
+    case KVC_OPT_BEACON_UPDATE_IMPL:
+      if (value < 0 || value > 2) return fail(ctx, KVC_ERR_INVALID_ARG, "impl must be 0, 1 or 2");
+      if (value == 2 && !beacon_update_tc_supported(ctx->cfg.head_dim, ctx->cfg.num_beacons, ctx->cfg.dtype))
+        return fail(ctx, KVC_ERR_UNSUPPORTED, "tcgen05 beacon update not available for this config");
+      ctx->update_impl = (int)value;
+      return KVC_OK;
   }
   return fail(ctx, KVC_ERR_INVALID_ARG, "unknown option");
 }
@@ -504,7 +511,10 @@ kvc_status kvc_update_beacons(kvc_ctx *ctx, int32_t *assign_out, float *ms_out) 
   p.d = c.head_dim;
   p.dtype = c.dtype;
   if (ms_out) KVC_CUDA(ctx, cudaEventRecord(ctx->ev[0], ctx->stream));
-  cudaError_t e = launch_beacon_update(p, (int)descs.size(), ctx->stream);
+  const bool use_tc = ctx->update_impl == 2 ||
+                      (ctx->update_impl == 0 && beacon_update_tc_supported(c.head_dim, B, c.dtype));
+  cudaError_t e = use_tc ? launch_beacon_update_tc(p, (int)descs.size(), ctx->stream)
+                         : launch_beacon_update(p, (int)descs.size(), ctx->stream);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "beacon_update");
   if (ms_out) KVC_CUDA(ctx, cudaEventRecord(ctx->ev[1], ctx->stream));
   if (kvc_status s = stage_release(ctx, st)) return s;

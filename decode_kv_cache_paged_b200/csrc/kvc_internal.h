@@ -97,5 +97,7 @@ cudaError_t launch_beacon_score_simt(const BeaconScoreParams &p, int n_req, cuda
 cudaError_t launch_beacon_score_tc(const BeaconScoreParams &p, int n_req, int max_l,
                                    cudaStream_t s);
 bool beacon_score_tc_supported(int d, int B, int dtype);
+cudaError_t launch_beacon_update_tc(const BeaconUpdateParams &p, int n_req, cudaStream_t s);
+bool beacon_update_tc_supported(int d, int B, int dtype);
 
 }  // namespace kvc

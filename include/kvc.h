@@ -143,7 +143,10 @@ typedef struct {
 } kvc_view;
 
 typedef enum {
-  KVC_OPT_BEACON_SCORE_IMPL = 0 /* 0 auto, 1 SIMT fp32 kernel, 2 tcgen05 (bf16 only) */
+  KVC_OPT_BEACON_SCORE_IMPL = 0, /* 0 auto, 1 SIMT fp32 kernel, 2 tcgen05 (bf16, head_dim 128) */
+  KVC_OPT_BEACON_UPDATE_IMPL = 1 /* 0 auto, 1 SIMT fp32 kernel, 2 tcgen05 assignment (bf16, head_dim 128,
+                                    B a multiple of 32): x.c as x.c_hi + x.c_lo with bf16 terms of the
+                                    fp32 beacons, error <= 2^-18 sum_k |x_k c_k| beyond fp32 rounding */
 } kvc_option;
 
 typedef struct kvc_ctx kvc_ctx;

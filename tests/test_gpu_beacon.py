@@ -174,3 +174,53 @@ def test_tcgen05_256_beacons():
     w.prompt = np.array([77])
     out = run_beacon(w, score_impl=2)
     print(out)
+
+
+@pytest.mark.parametrize("impl", [1, 2], ids=["simt", "tcgen05"])
+def test_second_update_against_oracle(impl):
+    """A later (non-initial) update: fp32 beacons with counts, new points.
+    The oracle recomputes it from the GPU's beacons and counts before the
+    update; assignments may differ only on near-ties within the kernels'
+    error bound (fp32 rounding, plus 2^-18 sum|x_k c_k| per dot product for
+    the tensor-core kernel's two-term bf16 split of the beacons)."""
+    w = wl.beacon_serving(R=2, layers=2)
+    ctx = make_context(w, headroom=256)
+    ctx.set_option(1, impl)
+    gen = wl.Generator(w, "cuda")
+    _fill_recording(ctx, w, gen)
+    ctx.update_beacons()
+    ctx.sync()
+    st = ctx.state_tensors()
+    c_before = st["beacons"].double().cpu().numpy()
+    n_before = st["beacon_counts"].cpu().numpy().astype(np.int64)
+    R, Ly, H, d, B, G, W = 2, 2, 8, 128, 64, 4, 64
+    q = gen.queries(R, W)
+    k, v = gen.kv(R, W)
+    ctx.append(np.arange(R, dtype=np.int32), k, v, q)
+    assign = torch.full((R, Ly, H, W * G), -1, dtype=torch.int32, device="cuda")
+    ctx.update_beacons(assign_out=assign)
+    ctx.sync()
+    g_beacons = st["beacons"].double().cpu().numpy()
+    g_counts = st["beacon_counts"].cpu().numpy()
+    g_assign = assign.cpu().numpy()
+    qn = q.float().cpu().numpy().astype(np.float64)  # [R, Ly, W, Hq, d]
+    ties = 0
+    for r in range(R):
+        for l in range(Ly):
+            for h in range(H):
+                pts = oracle.segment_points(qn[r, l], h, G)
+                c0 = c_before[r, l, h]
+                _, _, a_o = oracle.beacon_update(pts, c0, n_before[r, l, h], init=False)
+                ga = g_assign[r, l, h, :len(pts)]
+                for p in np.nonzero(a_o != ga)[0]:
+                    d_o = np.sum((pts[p] - c0[a_o[p]]) ** 2)
+                    d_g = np.sum((pts[p] - c0[ga[p]]) ** 2)
+                    bound = 4 * 2.0 ** -18 * max(np.abs(pts[p] * c0[a_o[p]]).sum(),
+                                                 np.abs(pts[p] * c0[ga[p]]).sum()) + 1e-5 * d_o
+                    assert d_g - d_o <= bound, (r, l, h, p, d_o, d_g, bound)
+                    ties += 1
+                c_s, cnt_s, _ = oracle.beacon_update(pts, c0, n_before[r, l, h], init=False, assign_override=ga)
+                assert np.array_equal(cnt_s, g_counts[r, l, h])
+                assert np.allclose(g_beacons[r, l, h], c_s, rtol=1e-5, atol=1e-6)
+    ctx.close()
+    print("near-tie assignments:", ties)
