@@ -22,7 +22,8 @@
 // Work in base 2: u = z_raw * log2(e)/sqrt(d), lse2 = log2 sum 2^u, score =
 // 2^(max_b u_bj - lse2_b).
 // Warp roles: warp 0 allocates TMEM and issues the TMA loads (one 2-D tiled
-// load per (page, 64-column half): a page holds 16 keys x 256 B contiguous,
+// load per (page, 64-column half), lane q of the warp taking page q of the
+// tile, page ids loaded one tile ahead: a page holds 16 keys x 256 B contiguous,
 // the tensor map covers the whole pool as rows of 128 bf16, 128-byte
 // swizzle); warp 1 issues the MMAs (one elected lane) and commits them to
 // mbarriers; warps 2-9 run the epilogue in two groups of four, group g taking
@@ -40,11 +41,17 @@
 #include "kvc_internal.h"
 #include "tc_ptx.cuh"
 
+#ifndef KVC_TC_NCB_SMALL
+#define KVC_TC_NCB_SMALL 2
+#endif
+#ifndef KVC_TC_STAGES_SMALL
+#define KVC_TC_STAGES_SMALL 4
+#endif
+
 namespace kvc {
 namespace {
 
 constexpr int kTileKeys = 128;
-constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;   // two groups of 4: group g drains accumulator buffer g
 constexpr int kThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr uint32_t kTmemCols = 512;
@@ -65,7 +72,17 @@ struct SegGeom {
   int r, l, h, L, P;
   int64_t seg_flat;
   int n1, t2, n2;  // pass-1 tiles, first pass-2 tile, pass-2 tiles
+  int nres;        // pass-2 tiles still resident in their pass-1 stages
+  // tile index of item t of the segment's sequence: pass 1 in order, then
+  // pass 2 starting with the resident tiles (the last nres of pass 1), then
+  // the remaining generated tiles in order
+  __device__ __forceinline__ int tile_of(int t) const {
+    if (t < n1) return t;
+    const int u = t - n1;
+    return u < nres ? n1 - nres + u : t2 + (u - nres);
+  }
 };
+template <int S>
 __device__ __forceinline__ SegGeom seg_geom(const TcParams &p, int s) {
   SegGeom g;
   g.h = s % p.hkv;
@@ -78,10 +95,13 @@ __device__ __forceinline__ SegGeom seg_geom(const TcParams &p, int s) {
   g.n1 = (g.L + kTileKeys - 1) / kTileKeys;
   g.t2 = g.P / kTileKeys;
   g.n2 = g.n1 - g.t2;
+  // item n1 + k lands in the stage that held pass-1 item n1 + k - S, i.e. the
+  // tile n1 - S + k, exactly when S pass-2 items reuse the last S pass-1 tiles
+  g.nres = (g.n1 >= S && g.n2 >= S) ? S : 0;
   return g;
 }
 
-template <int CROWS, int NCB>
+template <int CROWS, int NCB, int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
     beacon_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap cmap,
                            TcParams p) {
@@ -135,13 +155,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      uint32_t it = 0;  // key-tile counter across segments
-      int si = 0;       // local segment counter
-      for (int s = blockIdx.x; s < p.n_segs && !*abort_flag; s += gridDim.x, ++si) {
-        const SegGeom g = seg_geom(p, s);
-        const int cb = si % NCB;
-        if (!mbar_wait(&c_empty[cb], ((si / NCB) & 1) ^ 1, abort_flag, p.status)) break;
+    // The whole warp walks the tile sequence in step (waits by lane 0,
+    // results and the abort flag broadcast); lane q issues the two loads of
+    // page q of each tile, so a tile's 16 loads leave in one instruction.
+    constexpr int kTP = kTileKeys / kPage;
+    auto uniform_abort = [&]() { return __shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0) != 0; };
+    uint32_t it = 0;  // key-tile counter across segments
+    int si = 0;       // local segment counter
+    for (int s = blockIdx.x; s < p.n_segs; s += gridDim.x, ++si) {
+      if (uniform_abort()) break;
+      const SegGeom g = seg_geom<kStages>(p, s);
+      const int cb = si % NCB;
+      if (!warp_wait(&c_empty[cb], ((si / NCB) & 1) ^ 1, abort_flag, p.status)) break;
+      if (lane == 0) {
         mbar_expect_tx(&c_full[cb], (uint32_t)B * 256u * (dup ? 2u : 1u));
         const int crow = (int)(g.seg_flat * B);
         for (int copy = 0; copy < (dup ? 2 : 1); ++copy) {
@@ -149,30 +175,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(smem_u32(cdst), &cmap, 0, crow, &c_full[cb]);
           tma_load_2d(smem_u32(cdst + CROWS * 128), &cmap, 64, crow, &c_full[cb]);
         }
-        const int32_t *bt = p.block_table + (int64_t)g.r * p.bt_stride;
-        const int pages = (g.L + kPage - 1) / kPage;
-        for (int t = 0; t < g.n1 + g.n2 && !*abort_flag; ++t, ++it) {
-          const int tile = t < g.n1 ? t : g.t2 + (t - g.n1);
-          const int st = it % kStages;
-          if (!mbar_wait(&empty[st], ((it / kStages) & 1) ^ 1, abort_flag, p.status)) break;
-          const int pg0 = tile * (kTileKeys / kPage);
-          const int npg = min(kTileKeys / kPage, pages - pg0);
-          mbar_expect_tx(&full[st], (uint32_t)npg * 2u * 2048u);
-          uint8_t *dst = kbuf + st * kTileBytes;
-          for (int q = 0; q < npg; ++q) {
-            const int64_t row = (((int64_t)g.l * p.num_pages + bt[pg0 + q]) * p.hkv + g.h) * kPage;
-            tma_load_2d(smem_u32(dst + q * 2048), &kmap, 0, (int)row, &full[st]);
-            tma_load_2d(smem_u32(dst + kTileKeys * 128 + q * 2048), &kmap, 64, (int)row, &full[st]);
+      }
+      const int32_t *bt = p.block_table + (int64_t)g.r * p.bt_stride;
+      const int pages = (g.L + kPage - 1) / kPage;
+      // this lane's page id of a tile (lanes >= 8 idle), loaded one tile ahead
+      auto page_of = [&](int tile) { const int pg = tile * kTP + lane; return (lane < kTP && pg < pages) ? __ldg(bt + pg) : 0; };
+      int pg_cur = page_of(g.tile_of(0));
+      const int n_items = g.n1 + g.n2;
+      bool ok = true;
+      for (int t = 0; t < n_items; ++t, ++it) {
+        if (uniform_abort()) {
+          ok = false;
+          break;
+        }
+        const int tile = g.tile_of(t);
+        const int pg_next = (t + 1 < n_items) ? page_of(g.tile_of(t + 1)) : 0;
+        const int st = it % kStages;
+        if (!warp_wait(&empty[st], ((it / kStages) & 1) ^ 1, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        if (t >= g.n1 && t - g.n1 < g.nres) {
+          if (lane == 0) mbar_arrive(&full[st]);  // the tile is still in this stage from pass 1
+        } else {
+          const int npg = min(kTP, pages - tile * kTP);
+          if (lane == 0) mbar_expect_tx(&full[st], (uint32_t)npg * 2u * 2048u);
+          __syncwarp();
+          if (lane < npg) {
+            uint8_t *dst = kbuf + st * kTileBytes;
+            const int64_t row = (((int64_t)g.l * p.num_pages + pg_cur) * p.hkv + g.h) * kPage;
+            tma_load_2d(smem_u32(dst + lane * 2048), &kmap, 0, (int)row, &full[st]);
+            tma_load_2d(smem_u32(dst + kTileKeys * 128 + lane * 2048), &kmap, 64, (int)row, &full[st]);
           }
         }
+        __syncwarp();
+        pg_cur = pg_next;
       }
-      if (*abort_flag) {
-        // let loads already issued land before the CTA's shared memory goes away
-        for (int i = 0; i < kStages && it > 0; ++i) {
-          const uint32_t k = it - 1 - i;
-          mbar_wait(&full[k % kStages], (k / kStages) & 1, abort_flag, p.status, false);
-          if (k == 0) break;
-        }
+      if (!ok) break;
+    }
+    if (lane == 0 && *abort_flag) {
+      // let loads already issued land before the CTA's shared memory goes away
+      for (int i = 0; i < kStages && it > 0; ++i) {
+        const uint32_t k = it - 1 - i;
+        mbar_wait(&full[k % kStages], (k / kStages) & 1, abort_flag, p.status, false);
+        if (k == 0) break;
       }
     }
   } else if (warp == 1) {
@@ -184,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc2 = idesc_bf16_f32(128, B);
       bool ok = true;
       for (int s = blockIdx.x; s < p.n_segs && ok; s += gridDim.x, ++si) {
-        const SegGeom g = seg_geom(p, s);
+        const SegGeom g = seg_geom<kStages>(p, s);
         const int cb = si % NCB;
         ok = mbar_wait(&c_full[cb], (si / NCB) & 1, abort_flag, p.status);
         if (!ok) break;
@@ -240,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int si = 0;
     bool ok = true;
     for (int s = blockIdx.x; s < p.n_segs && ok; s += gridDim.x, ++si) {
-      const SegGeom g = seg_geom(p, s);
+      const SegGeom g = seg_geom<kStages>(p, s);
       float *lse_buf = lse2 + (si & 1) * 256;
       // pass 1: per-beacon online log2-sum-exp2 over this group's tiles
       float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
@@ -350,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        const int j = (g.t2 + t) * kTileKeys + row;
+        const int j = g.tile_of(g.n1 + t) * kTileKeys + row;
         if (j >= g.P && j < g.L) {
           const float best = fmaxf(fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3])),
                                    fmaxf(fmaxf(bm[4], bm[5]), fmaxf(bm[6], bm[7])));
@@ -394,18 +440,18 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int CROWS, int NCB>
+template <int CROWS, int NCB, int kStages>
 cudaError_t launch(const CUtensorMap &km, const CUtensorMap &cm, const TcParams &tp, cudaStream_t s) {
   const size_t smem = 1024 + (size_t)NCB * CROWS * 256 + (size_t)kStages * kTileKeys * 256 + 256 +
                       2 * 256 * 4 + 4 * 2 * 256 * 4;
-  cudaError_t e = cudaFuncSetAttribute(beacon_score_tc_kernel<CROWS, NCB>,
+  cudaError_t e = cudaFuncSetAttribute(beacon_score_tc_kernel<CROWS, NCB, kStages>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = tp.n_segs < sms ? tp.n_segs : sms;
-  beacon_score_tc_kernel<CROWS, NCB><<<grid, kThreads, smem, s>>>(km, cm, tp);
+  beacon_score_tc_kernel<CROWS, NCB, kStages><<<grid, kThreads, smem, s>>>(km, cm, tp);
   return cudaGetLastError();
 }
 
@@ -440,8 +486,8 @@ cudaError_t launch_beacon_score_tc(const BeaconScoreParams &p, int n_req, int ma
   tp.max_seq = p.max_seq;
   tp.n_segs = n_req * p.layers * p.hkv;
   tp.alpha = 1.4426950408889634f / sqrtf(128.0f);
-  if (p.B <= 128) return launch<128, 2>(km, cm, tp, s);
-  return launch<256, 1>(km, cm, tp, s);
+  if (p.B <= 128) return launch<128, KVC_TC_NCB_SMALL, KVC_TC_STAGES_SMALL>(km, cm, tp, s);
+  return launch<256, 1, 4>(km, cm, tp, s);
 }
 
 }  // namespace kvc
