@@ -176,14 +176,17 @@ def test_tcgen05_256_beacons():
     print(out)
 
 
-@pytest.mark.parametrize("impl", [1, 2], ids=["simt", "tcgen05"])
-def test_second_update_against_oracle(impl):
+@pytest.mark.parametrize("impl,B", [(1, 64), (2, 64), (2, 32), (2, 96), (2, 128), (2, 256)],
+                         ids=["simt-64", "tc-64", "tc-32", "tc-96", "tc-128", "tc-256"])
+def test_second_update_against_oracle(impl, B):
     """A later (non-initial) update: fp32 beacons with counts, new points.
     The oracle recomputes it from the GPU's beacons and counts before the
     update; assignments may differ only on near-ties within the kernels'
     error bound (fp32 rounding, plus 2^-18 sum|x_k c_k| per dot product for
     the tensor-core kernel's two-term bf16 split of the beacons)."""
     w = wl.beacon_serving(R=2, layers=2)
+    w.num_beacons = B
+    w.query_window = max(64, B // 4)  # the first update needs at least B points
     ctx = make_context(w, headroom=256)
     ctx.set_option(1, impl)
     gen = wl.Generator(w, "cuda")
@@ -193,11 +196,11 @@ def test_second_update_against_oracle(impl):
     st = ctx.state_tensors()
     c_before = st["beacons"].double().cpu().numpy()
     n_before = st["beacon_counts"].cpu().numpy().astype(np.int64)
-    R, Ly, H, d, B, G, W = 2, 2, 8, 128, 64, 4, 64
+    R, Ly, H, d, G, W = 2, 2, 8, 128, 4, 64
     q = gen.queries(R, W)
     k, v = gen.kv(R, W)
     ctx.append(np.arange(R, dtype=np.int32), k, v, q)
-    assign = torch.full((R, Ly, H, W * G), -1, dtype=torch.int32, device="cuda")
+    assign = torch.full((R, Ly, H, w.query_window * G), -1, dtype=torch.int32, device="cuda")
     ctx.update_beacons(assign_out=assign)
     ctx.sync()
     g_beacons = st["beacons"].double().cpu().numpy()
