@@ -22,7 +22,8 @@
 //      ballots gives every survivor its destination rank; the inverse map
 //      rank -> source slot is kept as uint16 in shared memory;
 //   4. copy: survivors from the first evicted slot on move to slot P + rank.
-//      Each chunk of ranks is read (16-byte vector loads, K and V rows plus
+//      Each chunk of ranks (8 rows per thread group, 64-128 KB of K and V in
+//      flight per CTA) is read (16-byte vector loads, K and V rows plus
 //      the position entry) into registers, the CTA synchronises, then writes.
 //      A chunk only writes slots below its own highest source slot, and the
 //      next chunk only reads slots above it, so one barrier per chunk makes
@@ -34,7 +35,12 @@
 namespace kvc {
 namespace {
 
-constexpr int kUnroll = 4;  // row passes per copy chunk
+#ifndef KVC_SC_UNROLL_SMALL
+#define KVC_SC_UNROLL_SMALL 8
+#endif
+#ifndef KVC_SC_UNROLL_LARGE
+#define KVC_SC_UNROLL_LARGE 8
+#endif
 
 __device__ __forceinline__ uint32_t float_order_key(float f) {
   const uint32_t u = __float_as_uint(f);
@@ -102,7 +108,7 @@ __device__ __forceinline__ void block_radix_select(const uint32_t *keys, int n, 
   need = k;
 }
 
-template <int NT, int MODE>
+template <int NT, int MODE, int kUnroll>
 __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams p, int keys_cap) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint32_t *keys = reinterpret_cast<uint32_t *>(smem);                  // [keys_cap]
@@ -228,7 +234,7 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
   if (tid == 0 && M > q0) atomicAdd(p.counters, (unsigned long long)(M - q0));
 }
 
-template <int NT>
+template <int NT, int U>
 cudaError_t launch_nt(const SelectCompactParams &p, int mode, int n_seg_req, int max_n,
                       cudaStream_t s) {
   const int keys_cap = (max_n + 7) & ~7;
@@ -237,22 +243,22 @@ cudaError_t launch_nt(const SelectCompactParams &p, int mode, int n_seg_req, int
   cudaError_t e = cudaSuccess;
   switch (mode) {
     case kModeRandom:
-      e = cudaFuncSetAttribute(select_compact_kernel<NT, kModeRandom>,
+      e = cudaFuncSetAttribute(select_compact_kernel<NT, kModeRandom, U>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e == cudaSuccess)
-        select_compact_kernel<NT, kModeRandom><<<grid, NT, smem, s>>>(p, keys_cap);
+        select_compact_kernel<NT, kModeRandom, U><<<grid, NT, smem, s>>>(p, keys_cap);
       break;
     case kModeRandomShared:
-      e = cudaFuncSetAttribute(select_compact_kernel<NT, kModeRandomShared>,
+      e = cudaFuncSetAttribute(select_compact_kernel<NT, kModeRandomShared, U>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e == cudaSuccess)
-        select_compact_kernel<NT, kModeRandomShared><<<grid, NT, smem, s>>>(p, keys_cap);
+        select_compact_kernel<NT, kModeRandomShared, U><<<grid, NT, smem, s>>>(p, keys_cap);
       break;
     default:
-      e = cudaFuncSetAttribute(select_compact_kernel<NT, kModeScores>,
+      e = cudaFuncSetAttribute(select_compact_kernel<NT, kModeScores, U>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e == cudaSuccess)
-        select_compact_kernel<NT, kModeScores><<<grid, NT, smem, s>>>(p, keys_cap);
+        select_compact_kernel<NT, kModeScores, U><<<grid, NT, smem, s>>>(p, keys_cap);
       break;
   }
   if (e != cudaSuccess) return e;
@@ -265,8 +271,8 @@ cudaError_t launch_select_compact(const SelectCompactParams &p, int mode, int n_
                                   int max_n, int max_m, cudaStream_t s) {
   (void)max_m;
   if (n_seg_req <= 0) return cudaSuccess;
-  if (max_n <= 4096) return launch_nt<256>(p, mode, n_seg_req, max_n, s);
-  return launch_nt<512>(p, mode, n_seg_req, max_n, s);
+  if (max_n <= 4096) return launch_nt<256, KVC_SC_UNROLL_SMALL>(p, mode, n_seg_req, max_n, s);
+  return launch_nt<512, KVC_SC_UNROLL_LARGE>(p, mode, n_seg_req, max_n, s);
 }
 
 }  // namespace kvc
