@@ -42,6 +42,9 @@ PINS = {
     "round_bf16": "torch fp32 -> bfloat16 conversion (round to nearest even)",
     "beacon_update": "scipy.cluster.vq.vq assignment; running mean == mean of assignment history",
     "beacon_score": "scipy.special.softmax; identical keys -> 1/L; B=1 ranking; one-hot closed form",
+    "random_score_block": "numpy.random.Philox on counter (pos // block, h, l, r)",
+    "hole_fill": "invariants: kept slots below R stay, holes filled in ascending order, same kept set",
+    "random_round_ex": "at most one split block; sink protection = prompt protection with P = S",
 }
 
 
@@ -82,6 +85,14 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.orc_beacon_update.restype = i32
     L.orc_beacon_score.argtypes = [i64, i64, i64, i64, P, P, P, P]
     L.orc_beacon_score.restype = i32
+    L.orc_random_score_block.argtypes = [u64, u64, i64, i64, i64, i64, i32, i64]
+    L.orc_random_score_block.restype = ctypes.c_uint32
+    L.orc_hole_fill.argtypes = [i64, P, P]
+    L.orc_hole_fill.restype = i64
+    L.orc_random_round_segment_ex.argtypes = [u64, u64, i64, i64, i64, i32, i64, i32, i64, i64, i64, P, P]
+    L.orc_random_round_segment_ex.restype = i64
+    L.orc_random_round_batch_ex.argtypes = [u64, u64, i32, i64, i32, i64, P, P, i64, P, P, P]
+    L.orc_random_round_batch_ex.restype = i64
     return L
 
 
@@ -217,6 +228,45 @@ def random_round_batch(seed, rnd, shared, rlh, lpk, pos_in):
                                       _ptr(pos_in), _ptr(pos_out), _ptr(R))
     if rc != 0:
         raise ValueError(f"random_round_batch failed at segment {rc - 1}")
+    return pos_out, R
+
+
+def random_score_block(seed, rnd, r, l, h, pos, shared=False, block=1) -> int:
+    return int(lib().orc_random_score_block(seed, rnd, r, l, h, pos, int(bool(shared)), block))
+
+
+def hole_fill(R: int, kept_slots) -> np.ndarray:
+    """For each new slot s < R, the old slot whose row it holds after hole filling."""
+    kept = np.ascontiguousarray(kept_slots, dtype=np.int64)
+    out = np.zeros(max(R, 1), np.int64)
+    if lib().orc_hole_fill(R, _ptr(kept), _ptr(out)) < 0:
+        raise ValueError("hole_fill failed")
+    return out[:R]
+
+
+def random_round_segment_ex(seed, rnd, r, l, h, shared, block, hole_fill_mode, P, K, pos_in):
+    """pos_out [R] of one segment under the extended round's options."""
+    pos_in = np.ascontiguousarray(pos_in, dtype=np.int32)
+    L = len(pos_in)
+    pos_out = np.zeros(max(L, 1), np.int32)
+    R = lib().orc_random_round_segment_ex(seed, rnd, r, l, h, int(bool(shared)), block,
+                                          int(bool(hole_fill_mode)), L, P, K, _ptr(pos_in), _ptr(pos_out))
+    if R < 0:
+        raise ValueError("random_round_segment_ex failed")
+    return pos_out[:R]
+
+
+def random_round_batch_ex(seed, rnd, shared, block, hole_fill_mode, rlh, lpk, pos_in):
+    rlh = np.ascontiguousarray(rlh, dtype=np.int64)
+    lpk = np.ascontiguousarray(lpk, dtype=np.int64)
+    pos_in = np.ascontiguousarray(pos_in, dtype=np.int32)
+    n, stride = pos_in.shape
+    pos_out = np.full((n, stride), -1, np.int32)
+    R = np.zeros(n, np.int64)
+    rc = lib().orc_random_round_batch_ex(seed, rnd, int(bool(shared)), block, int(bool(hole_fill_mode)), n,
+                                         _ptr(rlh), _ptr(lpk), stride, _ptr(pos_in), _ptr(pos_out), _ptr(R))
+    if rc != 0:
+        raise ValueError(f"random_round_batch_ex failed at segment {rc - 1}")
     return pos_out, R
 
 

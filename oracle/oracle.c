@@ -102,6 +102,18 @@ uint32_t orc_random_score(uint64_t seed, uint64_t round, int64_t r, int64_t l, i
   return (uint32_t)(out[0] >> 32);
 }
 
+/* Block-granular variant [RA, "发现二": retaining contiguous blocks of 1 to
+ * 256 tokens instead of scattered ones]: every original position of a block
+ * of `block` consecutive positions (block index pos / block) shares one draw,
+ * so Top-K keeps whole blocks in order of their draw; ties, i.e. positions of
+ * one block, go to the lower position, so at most one block is split.
+ * Reading: blocks are aligned to multiples of `block` in original-position
+ * space; block = 1 is the per-token score. */
+uint32_t orc_random_score_block(uint64_t seed, uint64_t round, int64_t r, int64_t l, int64_t h,
+                                int64_t pos, int32_t shared, int64_t block) {
+  return orc_random_score(seed, round, r, l, h, pos / (block > 0 ? block : 1), shared);
+}
+
 /* ------------------------------------------------------------------ */
 /* Retention rule [RA, "长推理的显存瓶颈" and "Random Attention：..."]. */
 /* ------------------------------------------------------------------ */
@@ -237,6 +249,85 @@ int64_t orc_random_round_segment(uint64_t seed, uint64_t round, int64_t r, int64
   return R;
 }
 
+/* Hole-filling compaction (the build's option; the pages only require
+ * "cache compaction"): the kept slots below the new length R stay where they
+ * are, and the kept slots at or above R fill the evicted slots below R, the
+ * i-th such hole (ascending) taking the i-th such survivor (ascending).
+ * kept_slots[0..R) ascending on input; slot_out[0..R) receives, for each new
+ * slot s, the old slot whose row it holds.  Returns the number of moves. */
+int64_t orc_hole_fill(int64_t R, const int64_t *kept_slots, int64_t *slot_out) {
+  int64_t n_hole = 0, n_move = 0, next_hole_search = 0;
+  for (int64_t s = 0; s < R; ++s) slot_out[s] = -1;
+  for (int64_t i = 0; i < R; ++i)
+    if (kept_slots[i] < R) slot_out[kept_slots[i]] = kept_slots[i];
+  for (int64_t i = 0; i < R; ++i) {
+    if (kept_slots[i] < R) continue;
+    while (next_hole_search < R && slot_out[next_hole_search] >= 0) ++next_hole_search;
+    slot_out[next_hole_search] = kept_slots[i];
+    ++n_move;
+  }
+  for (int64_t s = 0; s < R; ++s)
+    if (slot_out[s] < 0) ++n_hole;
+  return n_hole == 0 ? n_move : -1;
+}
+
+/* One random round with the options of the extended round: protection of
+ * the first `protect` positions only (sink tokens) instead of the whole
+ * prompt, block-granular draws, hole-filling compaction.  pos_in[0..L);
+ * writes pos_out[0..R) and returns R (or -1). */
+int64_t orc_random_round_segment_ex(uint64_t seed, uint64_t round, int64_t r, int64_t l, int64_t h,
+                                    int32_t shared, int64_t block, int32_t hole_fill, int64_t L,
+                                    int64_t P, int64_t K, const int32_t *pos_in, int32_t *pos_out) {
+  int64_t M, R;
+  int32_t flags;
+  if (orc_retention(L, P, K, &M, &R, &flags) != 0) return -1;
+  int64_t *kept = (int64_t *)malloc((size_t)(L > 0 ? L : 1) * sizeof(int64_t));
+  if (!kept) return -1;
+  for (int64_t s = 0; s < P; ++s) kept[s] = s;
+  if (flags & 1) {
+    for (int64_t s = P; s < L; ++s) kept[s] = s;
+  } else if (M > 0) {
+    int64_t N = L - P;
+    double *score = (double *)malloc((size_t)N * sizeof(double));
+    int64_t *pos = (int64_t *)malloc((size_t)N * sizeof(int64_t));
+    int64_t *slot = (int64_t *)malloc((size_t)N * sizeof(int64_t));
+    if (!score || !pos || !slot) {
+      free(score);
+      free(pos);
+      free(slot);
+      free(kept);
+      return -1;
+    }
+    for (int64_t j = 0; j < N; ++j) {
+      slot[j] = P + j;
+      pos[j] = pos_in[P + j];
+      score[j] = (double)orc_random_score_block(seed, round, r, l, h, pos[j], shared, block);
+    }
+    int64_t got = orc_select_topk(N, score, pos, slot, M, kept + P);
+    free(score);
+    free(pos);
+    free(slot);
+    if (got != M) {
+      free(kept);
+      return -1;
+    }
+  }
+  if (hole_fill && !(flags & 1)) {
+    int64_t *src = (int64_t *)malloc((size_t)(R > 0 ? R : 1) * sizeof(int64_t));
+    if (!src || orc_hole_fill(R, kept, src) < 0) {
+      free(src);
+      free(kept);
+      return -1;
+    }
+    for (int64_t i = 0; i < R; ++i) pos_out[i] = pos_in[src[i]];
+    free(src);
+  } else {
+    for (int64_t i = 0; i < R; ++i) pos_out[i] = pos_in[kept[i]];
+  }
+  free(kept);
+  return R;
+}
+
 /* Batched form of orc_random_round_segment over n segments, for speed of the
  * test harness only (each segment is still processed by the plain routine).
  * rlh[3*s..] = (r, l, h); lpk[3*s..] = (L, P, K); pos_in/pos_out are
@@ -259,6 +350,23 @@ int64_t orc_random_round_batch(uint64_t seed, uint64_t round, int32_t shared, in
     for (int64_t i = R; i < stride; ++i) pos_out[s * stride + i] = -1;
   }
   free(kept);
+  return 0;
+}
+
+/* Batched orc_random_round_segment_ex; lpk[3*s..] = (L, P, K) with P the
+ * protected length actually used (the sink count under sink protection). */
+int64_t orc_random_round_batch_ex(uint64_t seed, uint64_t round, int32_t shared, int64_t block,
+                                  int32_t hole_fill, int64_t n, const int64_t *rlh,
+                                  const int64_t *lpk, int64_t stride, const int32_t *pos_in,
+                                  int32_t *pos_out, int64_t *R_out) {
+  for (int64_t s = 0; s < n; ++s) {
+    int64_t R = orc_random_round_segment_ex(seed, round, rlh[3 * s], rlh[3 * s + 1], rlh[3 * s + 2],
+                                            shared, block, hole_fill, lpk[3 * s], lpk[3 * s + 1],
+                                            lpk[3 * s + 2], pos_in + s * stride, pos_out + s * stride);
+    if (R < 0) return s + 1;
+    R_out[s] = R;
+    for (int64_t i = R; i < stride; ++i) pos_out[s * stride + i] = -1;
+  }
   return 0;
 }
 

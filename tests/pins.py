@@ -260,6 +260,59 @@ def check_beacon_score():
     assert np.allclose(sc, want, rtol=1e-13)
 
 
+def check_block_score():
+    rng = np.random.default_rng(13)
+    for _ in range(40):
+        seed, rnd = int(rng.integers(0, 2**40)), int(rng.integers(0, 100))
+        r, l, h, pos = (int(x) for x in rng.integers(0, 5000, 4))
+        block = int(rng.choice([1, 2, 16, 64, 256]))
+        for shared in (False, True):
+            want = numpy_philox_block([pos // block, U64 if shared else h, l, r], [seed, rnd])[0] >> 32
+            assert oracle.random_score_block(seed, rnd, r, l, h, pos, shared, block) == want
+
+
+def check_hole_fill():
+    rng = np.random.default_rng(17)
+    for _ in range(200):
+        L = int(rng.integers(1, 80))
+        R = int(rng.integers(0, L + 1))
+        kept = np.sort(rng.choice(L, R, replace=False)).astype(np.int64)
+        src = oracle.hole_fill(R, kept)
+        assert sorted(src.tolist()) == kept.tolist()            # same rows survive
+        for s in kept[kept < R]:
+            assert src[s] == s                                   # survivors below R stay
+        holes = [s for s in range(R) if s not in set(kept.tolist())]
+        movers = kept[kept >= R].tolist()
+        assert [int(src[s]) for s in holes] == movers            # holes in order take movers in order
+
+
+def check_random_round_ex():
+    rng = np.random.default_rng(19)
+    P, K, L = 16, 64, 256
+    pos_in = (np.arange(L) * 2 + 5).astype(np.int32)
+    for trial in range(30):
+        seed, rnd, h = int(rng.integers(0, 2**32)), int(rng.integers(0, 50)), int(rng.integers(0, 8))
+        # block 1, ordered: the pinned per-token round
+        want = oracle.random_round_segment(seed, rnd, 3, 2, h, False, P, K, pos_in)[1]
+        assert np.array_equal(oracle.random_round_segment_ex(seed, rnd, 3, 2, h, False, 1, False, P, K, pos_in), want)
+        # hole filling keeps the same positions; those already below R stay put
+        hf = oracle.random_round_segment_ex(seed, rnd, 3, 2, h, False, 1, True, P, K, pos_in)
+        assert sorted(hf.tolist()) == sorted(want.tolist())
+        for s in range(K):
+            if pos_in[s] in set(want.tolist()):
+                assert hf[s] == pos_in[s]
+        # block-granular draws split at most one block of candidates
+        for block in (4, 16, 64):
+            out = oracle.random_round_segment_ex(seed, rnd, 3, 2, h, False, block, False, P, K, pos_in)
+            kept = set(out.tolist())
+            blocks = {}
+            for pos in pos_in[P:]:
+                blocks.setdefault(int(pos) // block, []).append(int(pos) in kept)
+            split = sum(1 for v in blocks.values() if any(v) and not all(v))
+            assert split <= 1, (block, split)
+            assert len(out) == K and np.array_equal(out[:P], pos_in[:P])
+
+
 ALL = [check_philox, check_random_score, check_retention, check_select, check_compact,
        check_random_round_invariants, check_survival, check_head_independence, check_bf16,
-       check_beacon_update, check_beacon_score]
+       check_beacon_update, check_beacon_score, check_block_score, check_hole_fill, check_random_round_ex]

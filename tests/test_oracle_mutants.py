@@ -43,6 +43,11 @@ MUTANTS = [
      [pins.check_bf16]),
     ("bf16_truncates", "double q = nearbyint(ldexp(m, 8));", "double q = trunc(ldexp(m, 8));",
      [pins.check_bf16]),
+    ("block_index_modulo", "return orc_random_score(seed, round, r, l, h, pos / (block > 0 ? block : 1), shared);",
+     "return orc_random_score(seed, round, r, l, h, pos % (block > 0 ? block : 1), shared);",
+     [pins.check_block_score]),
+    ("hole_fill_reverse", "for (int64_t i = 0; i < R; ++i) {\n    if (kept_slots[i] < R) continue;",
+     "for (int64_t i = R - 1; i >= 0; --i) {\n    if (kept_slots[i] < R) continue;", [pins.check_hole_fill]),
 ]
 
 
