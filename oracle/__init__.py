@@ -45,6 +45,9 @@ PINS = {
     "random_score_block": "numpy.random.Philox on counter (pos // block, h, l, r)",
     "hole_fill": "invariants: kept slots below R stay, holes filled in ascending order, same kept set",
     "random_round_ex": "at most one split block; sink protection = prompt protection with P = S",
+    "decode_attention": "scipy.special.softmax/logsumexp; L=1 -> v; q=0 -> mean of v, log L; "
+                        "large-scale limit -> v of the argmax key; joint permutation invariance",
+    "decode_attention_gqa": "query head hq reads KV head hq // G (marker values per KV head)",
 }
 
 
@@ -93,6 +96,10 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.orc_random_round_segment_ex.restype = i64
     L.orc_random_round_batch_ex.argtypes = [u64, u64, i32, i64, i32, i64, P, P, i64, P, P, P]
     L.orc_random_round_batch_ex.restype = i64
+    L.orc_decode_attention.argtypes = [i64, i64, P, P, P, ctypes.c_double, P, P]
+    L.orc_decode_attention.restype = None
+    L.orc_decode_attention_gqa.argtypes = [i64, i64, i64, i64, P, P, P, ctypes.c_double, P, P]
+    L.orc_decode_attention_gqa.restype = None
     return L
 
 
@@ -343,3 +350,32 @@ def beacon_select_with_pos(scores32, pos, P: int, K: int):
     kept = select_topk(np.asarray(scores32, np.float32).astype(np.float64),
                        np.asarray(pos[P:], np.int64), slots, ret.M)
     return np.concatenate([np.arange(P, dtype=np.int64), kept])
+
+
+def decode_attention(q, k, v, scale=None):
+    """out [d], lse of one query over rows k, v [L, d] (float64)."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64).reshape(-1, q.shape[0])
+    v = np.ascontiguousarray(v, dtype=np.float64).reshape(-1, q.shape[0])
+    d = q.shape[0]
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    out = np.zeros(d, np.float64)
+    lse = np.zeros(1, np.float64)
+    lib().orc_decode_attention(k.shape[0], d, _ptr(q), _ptr(k), _ptr(v), scale, _ptr(out), _ptr(lse))
+    return out, float(lse[0])
+
+
+def decode_attention_gqa(q, k, v, scale=None):
+    """out [Hq, d], lse [Hq] for q [Hq, d] over k, v [Hkv, L, d] (float64)."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    Hq, d = q.shape
+    Hkv, L = k.shape[0], k.shape[1]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    out = np.zeros((Hq, d), np.float64)
+    lse = np.zeros(Hq, np.float64)
+    lib().orc_decode_attention_gqa(Hq, Hkv, L, d, _ptr(q), _ptr(k), _ptr(v), scale, _ptr(out), _ptr(lse))
+    return out, lse

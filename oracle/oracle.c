@@ -18,7 +18,8 @@
  *        "长推理的显存瓶颈" (fixed budget K), "Random Attention：不判断重要性，
  *        只随机保留" (prompt protection, per-head random Top-K, geometric
  *        survival), "发现二" (all heads sharing one random set) and
- *        "发现四" (cache compaction needed by every method).
+ *        "发现四" (cache compaction needed by every method; the paged
+ *        attention kernels every selector shares).
  *  [BX]  "BeaconKV: 用"信标查询"指导 KV cache 压缩 ..." explainer
  *        (papers.ananclaw.com/promo/explainers__2609-04971), §3.2 (nearest
  *        beacon assignment, periodic incremental beacon update).
@@ -514,4 +515,60 @@ int32_t orc_beacon_score(int64_t L, int64_t P, int64_t B, int64_t d, const doubl
   free(z);
   free(lse);
   return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Decode attention over a request's cached rows [RA, "发现四": every     */
+/* selector shares the same paged attention kernels; what they attend  */
+/* to is the compacted cache].                                         */
+/* ------------------------------------------------------------------ */
+
+/* Scaled dot-product attention of one decode query over L cached rows:
+ *     s_j = scale * (q . k_j),  j < L
+ *     out = sum_j exp(s_j - lse) v_j,  lse = log sum_j exp(s_j)
+ * (lse computed as max + log sum exp(s - max)).  q [d], k [L][d],
+ * v [L][d]; out [d].  L = 0 gives out = 0 and lse = -inf. */
+void orc_decode_attention(int64_t L, int64_t d, const double *q, const double *k, const double *v,
+                          double scale, double *out, double *lse_out) {
+  for (int64_t c = 0; c < d; ++c) out[c] = 0.0;
+  if (L <= 0) {
+    *lse_out = -INFINITY;
+    return;
+  }
+  double *s = (double *)malloc((size_t)L * sizeof(double));
+  if (!s) {
+    *lse_out = NAN;
+    return;
+  }
+  double mx = -INFINITY;
+  for (int64_t j = 0; j < L; ++j) {
+    double dot = 0.0;
+    for (int64_t c = 0; c < d; ++c) dot += q[c] * k[j * d + c];
+    s[j] = scale * dot;
+    if (s[j] > mx) mx = s[j];
+  }
+  double sum = 0.0;
+  for (int64_t j = 0; j < L; ++j) sum += exp(s[j] - mx);
+  double lse = mx + log(sum);
+  for (int64_t j = 0; j < L; ++j) {
+    double w = exp(s[j] - lse);
+    for (int64_t c = 0; c < d; ++c) out[c] += w * v[j * d + c];
+  }
+  *lse_out = lse;
+  free(s);
+}
+
+/* Grouped-query form for one (request, layer): Hq query heads over Hkv
+ * key/value heads, G = Hq / Hkv consecutive query heads per KV head (query
+ * head hq reads KV head hq / G, the grouping the beacon update uses for its
+ * points).  q [Hq][d], k and v [Hkv][L][d], out [Hq][d], lse [Hq]. */
+void orc_decode_attention_gqa(int64_t Hq, int64_t Hkv, int64_t L, int64_t d, const double *q,
+                              const double *k, const double *v, double scale, double *out,
+                              double *lse) {
+  int64_t G = Hq / Hkv;
+  for (int64_t hq = 0; hq < Hq; ++hq) {
+    int64_t h = hq / G;
+    orc_decode_attention(L, d, q + hq * d, k + h * L * d, v + h * L * d, scale, out + hq * d,
+                         lse + hq);
+  }
 }

@@ -313,6 +313,57 @@ def check_random_round_ex():
             assert len(out) == K and np.array_equal(out[:P], pos_in[:P])
 
 
+def check_decode_attention():
+    from scipy.special import logsumexp, softmax
+    rng = np.random.default_rng(23)
+    for (L, d, scale) in [(1, 8, None), (37, 16, None), (200, 64, 0.3), (5, 128, 2.0)]:
+        q = rng.standard_normal(d)
+        k = rng.standard_normal((L, d))
+        v = rng.standard_normal((L, d))
+        sc = 1 / np.sqrt(d) if scale is None else scale
+        out, lse = oracle.decode_attention(q, k, v, scale)
+        s = sc * (k @ q)
+        assert np.allclose(out, softmax(s) @ v, rtol=1e-12, atol=1e-14)
+        assert abs(lse - logsumexp(s)) <= 1e-12 * max(1.0, abs(lse))
+        # joint permutation of the rows changes nothing
+        perm = rng.permutation(L)
+        out2, lse2 = oracle.decode_attention(q, k[perm], v[perm], scale)
+        assert np.allclose(out2, out, rtol=1e-12, atol=1e-14) and abs(lse2 - lse) <= 1e-12 * max(1.0, abs(lse))
+    # one row: the value row itself, lse = the score
+    q, k, v = rng.standard_normal(8), rng.standard_normal((1, 8)), rng.standard_normal((1, 8))
+    out, lse = oracle.decode_attention(q, k, v)
+    assert np.array_equal(out, v[0]) and abs(lse - (k[0] @ q) / np.sqrt(8)) <= 1e-15
+    # zero query: the mean of the values, lse = log L
+    v = rng.standard_normal((50, 16))
+    out, lse = oracle.decode_attention(np.zeros(16), rng.standard_normal((50, 16)), v)
+    assert np.allclose(out, v.mean(0), rtol=1e-12, atol=1e-15) and abs(lse - np.log(50)) <= 1e-13
+    # large scale: all weight on the best key (no overflow)
+    k = rng.standard_normal((20, 16))
+    q = rng.standard_normal(16)
+    v = rng.standard_normal((20, 16))
+    out, lse = oracle.decode_attention(q, k, v, scale=1e4)
+    j = int(np.argmax(k @ q))
+    assert np.allclose(out, v[j], rtol=1e-9, atol=1e-12) and np.isfinite(lse)
+    # empty: zeros and -inf
+    out, lse = oracle.decode_attention(np.ones(4), np.zeros((0, 4)), np.zeros((0, 4)))
+    assert np.array_equal(out, np.zeros(4)) and lse == -np.inf
+
+
+def check_decode_attention_gqa():
+    rng = np.random.default_rng(29)
+    Hq, Hkv, L, d = 8, 2, 30, 16
+    q = rng.standard_normal((Hq, d))
+    k = rng.standard_normal((Hkv, L, d))
+    v = np.stack([np.full((L, d), 3.0), np.full((L, d), 7.0)])  # marker value per KV head
+    out, lse = oracle.decode_attention_gqa(q, k, v)
+    G = Hq // Hkv
+    for hq in range(Hq):
+        assert np.allclose(out[hq], 3.0 if hq // G == 0 else 7.0, rtol=1e-13)
+        s = k[hq // G] @ q[hq] / np.sqrt(d)
+        assert abs(lse[hq] - np.log(np.exp(s).sum())) <= 1e-12 * abs(lse[hq]) + 1e-13
+
+
 ALL = [check_philox, check_random_score, check_retention, check_select, check_compact,
        check_random_round_invariants, check_survival, check_head_independence, check_bf16,
-       check_beacon_update, check_beacon_score, check_block_score, check_hole_fill, check_random_round_ex]
+       check_beacon_update, check_beacon_score, check_block_score, check_hole_fill, check_random_round_ex,
+       check_decode_attention, check_decode_attention_gqa]

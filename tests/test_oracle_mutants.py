@@ -48,6 +48,13 @@ MUTANTS = [
      [pins.check_block_score]),
     ("hole_fill_reverse", "for (int64_t i = 0; i < R; ++i) {\n    if (kept_slots[i] < R) continue;",
      "for (int64_t i = R - 1; i >= 0; --i) {\n    if (kept_slots[i] < R) continue;", [pins.check_hole_fill]),
+    ("attention_no_scale", "s[j] = scale * dot;", "s[j] = dot;", [pins.check_decode_attention]),
+    ("attention_lse_drops_max", "double lse = mx + log(sum);", "double lse = log(sum);",
+     [pins.check_decode_attention]),
+    ("attention_weight_no_norm", "double w = exp(s[j] - lse);", "double w = exp(s[j] - mx);",
+     [pins.check_decode_attention]),
+    ("attention_gqa_modulo", "int64_t h = hq / G;", "int64_t h = hq % Hkv;", [pins.check_decode_attention_gqa]),
+    ("attention_value_row", "out[c] += w * v[j * d + c];", "out[c] += w * v[c];", [pins.check_decode_attention]),
 ]
 
 
