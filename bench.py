@@ -58,6 +58,14 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--score-impl", type=int, default=0, help="beacon score kernel: 0 auto, 1 SIMT, 2 tcgen05")
+    ap.add_argument("--compaction", default="ordered", choices=["ordered", "hole_fill"],
+                    help="round option: order-preserving or hole-filling compaction")
+    ap.add_argument("--block", type=int, default=1, help="round option: positions per Philox draw")
+    ap.add_argument("--sinks", type=int, default=None, help="round option: protect only this many sinks")
+    ap.add_argument("--phase", default="round", choices=["round", "attention"],
+                    help="round: the eviction round; attention: one decode step of attention over the "
+                         "compacted cache (all layers)")
+    ap.add_argument("--q-heads", type=int, default=32, help="query heads for --phase attention")
     return ap.parse_args()
 
 
@@ -268,12 +276,14 @@ def run_ours(args, rank, world, dist):
     T = w.trigger
     refill = Refill(ctx, w, gen)
 
+    opts = {"sink_tokens": args.sinks, "block": args.block, "compaction": args.compaction}
+
     def one_round(seed, timed):
         ev0 = torch.cuda.Event(enable_timing=True)
         ev1 = torch.cuda.Event(enable_timing=True)
         ev0.record(ctx.stream)
         upd_ms = ctx.update_beacons(timed=timed) if beacon else 0.0
-        st = ctx.compress(sel, budgets, seed, stats=timed)
+        st = ctx.compress(sel, budgets, seed, stats=timed, **opts)
         ev1.record(ctx.stream)
         return ev0, ev1, st, upd_ms
 
@@ -282,7 +292,7 @@ def run_ours(args, rank, world, dist):
     for i in range(args.warmup):
         if beacon:
             ctx.update_beacons()
-        ctx.compress(sel, budgets, w.philox_seed)
+        ctx.compress(sel, budgets, w.philox_seed, **opts)
         refill()
     torch.cuda.synchronize()
     if dist:
@@ -309,6 +319,10 @@ def run_ours(args, rank, world, dist):
 
     # roofline of the dominant kernel
     peaks, peak_kind = measured_peaks()
+    variant = [] if args.compaction == "ordered" else [args.compaction]
+    variant += [f"block{args.block}"] if args.block != 1 else []
+    variant += [f"sinks{args.sinks}"] if args.sinks is not None else []
+    traffic_key = "/".join([w.name] + variant)
     sc_ms = statistics.mean(s["ms_select_compact"] for s in stats)
     score_ms = statistics.mean(s["ms_score"] for s in stats)
     moved = statistics.mean(s["moved_rows"] for s in stats)
@@ -337,7 +351,7 @@ def run_ours(args, rank, world, dist):
     else:
         roof = {"kernel": "select_compact", "bound": "hbm", "achieved": sc_bytes / (sc_ms / 1e3) / 1e9,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "traffic": profiled_traffic("select_compact", w.name, moved)}
+                "traffic": profiled_traffic("select_compact", traffic_key, moved)}
     roof["frac"] = roof["achieved"] / roof["peak"] if roof.get("peak") else None
     roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})"
     roof["algorithmic_bytes_per_launch"] = sc_bytes if roof["kernel"] == "select_compact" else None
@@ -362,7 +376,7 @@ def run_ours(args, rank, world, dist):
             a.record(ctx.stream)
             if beacon:
                 ctx.update_beacons()
-            ctx.compress(sel, budgets, w.philox_seed)
+            ctx.compress(sel, budgets, w.philox_seed, **opts)
             len_h.copy_(lens_dev, non_blocking=True)
             ctx.append(ids, k_h, v_h, q_h)
             b.record(ctx.stream)
@@ -387,11 +401,14 @@ def run_ours(args, rank, world, dist):
                    "prompt": int(w.prompt[0]) if len(set(w.prompt.tolist())) == 1 else "ragged",
                    "budget": int(w.budget[0]) if len(set(w.budget.tolist())) == 1 else "ragged",
                    "trigger": T, "beacons": w.num_beacons, "page_size": 16,
+                   "compaction": args.compaction, "block": args.block,
+                   "sinks": "whole prompt" if args.sinks is None else args.sinks,
                    "head_positions_per_round_per_gpu": head_pos,
                    "parallelism": f"replicas x{world} (no collective on the data path)",
                    "l2": "inputs larger than L2: the cache is tens of GB vs 126 MB L2, and each "
                          "trigger append between rounds writes >1 GB"},
         "roofline": roof,
+        "moved_rows_per_round": [int(s["moved_rows"]) for s in stats],
         "phases_ms": {"select_compact": sc_ms, "score": score_ms, "update": statistics.mean(upd) if beacon else 0.0},
         "e2e": e2e,
         "gpu_launches": launches,
@@ -399,6 +416,152 @@ def run_ours(args, rank, world, dist):
         "wall_s_timed_region": wall,
     }
     return out, w, sel
+
+
+# ---------------------------------------------------- attention phase ---
+
+ATTN_METRIC = "cached head-positions attended/s per decode step"
+
+
+def attention_workload(args):
+    w, _ = make_workload(args)
+    wl = load_workloads()
+    if args.q_heads % w.num_kv_heads:
+        raise SystemExit("--q-heads must be a multiple of the KV heads")
+    return wl.scaled(w, num_beacons=0, query_window=0, num_q_heads=args.q_heads)
+
+
+def run_attention(args, rank, world, dist):
+    """One decode step of attention over every layer of the cache right after
+    an eviction round (lengths at the budget K), per timed step."""
+    import numpy as np
+    import torch
+
+    from decode_kv_cache_paged_b200 import workloads as wl
+    from decode_kv_cache_paged_b200 import Context, ContextSpec
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = attention_workload(args)
+    w.data_seed += 7 * rank
+    spec = ContextSpec(num_requests=w.num_requests, num_layers=w.num_layers, num_kv_heads=w.num_kv_heads,
+                       head_dim=w.head_dim, max_seq_len=w.max_seq_len(0),
+                       num_pages=w.pages_needed(0) + w.num_requests, num_q_heads=w.num_q_heads,
+                       num_beacons=0, query_window=0)
+    ctx = Context(spec, dtype=wl.torch_dtype(w.dtype), device=dev)
+    gen = wl.Generator(w, dev)
+    wl.fill(ctx, w, gen, with_queries=False)
+    ctx.compress("random", w.budget.astype(np.int32), w.philox_seed)
+    lengths, _ = ctx.lengths()
+    positions = int(lengths.sum()) * w.num_layers * w.num_kv_heads
+    g = torch.Generator(device=dev).manual_seed(1 + rank)
+    q = torch.randn((w.num_layers, w.num_requests, w.num_q_heads, w.head_dim), generator=g, device=dev)
+    q = q.to(ctx.dtype)
+    out = torch.empty((w.num_layers, w.num_requests, w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.num_layers, w.num_requests, w.num_q_heads), dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        ctx.decode_attention(q, out=out, lse=lse)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clock = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    clock.start()
+    evs = []
+    for _ in range(args.steps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(ctx.stream)
+        ctx.decode_attention(q, out=out, lse=lse)
+        b.record(ctx.stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = clock.stop()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    value, total_ms = aggregate(sum(ms), positions, args.steps, world, dist, dev)
+    peaks, peak_kind = measured_peaks()
+    rb = w.head_dim * (2 if w.dtype == "bf16" else 4)
+    io_bytes = q.numel() * q.element_size() + out.numel() * 4 + lse.numel() * 4
+    alg_bytes = positions * rb * 2 + io_bytes
+    mean_ms = statistics.mean(ms)
+    roof = {"kernel": "decode_attention", "bound": "hbm", "achieved": alg_bytes / (mean_ms / 1e3) / 1e9,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "traffic": None,
+            "peak_source": f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})",
+            "algorithmic_bytes_per_launch": alg_bytes, "launch_ms": mean_ms}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    e2e = None
+    if not args.no_e2e:
+        q_h = q.cpu().pin_memory()
+        out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        times = []
+        for i in range(args.e2e_steps + 1):
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(ctx.stream)
+            with torch.cuda.stream(ctx.stream):
+                q.copy_(q_h, non_blocking=True)
+            ctx.decode_attention(q, out=out, lse=lse)
+            with torch.cuda.stream(ctx.stream):
+                out_h.copy_(out, non_blocking=True)
+            b.record(ctx.stream)
+            b.synchronize()
+            if i > 0:
+                times.append(a.elapsed_time(b))
+        e2e_value, e2e_ms = aggregate(statistics.mean(times), positions, 1, world, dist, dev)
+        e2e = {"value": e2e_value, "unit": "head-positions/s", "h2d_bytes_per_step": int(q_h.numel() * q_h.element_size()),
+               "d2h_bytes_per_step": int(out_h.numel() * 4), "ms_per_step": e2e_ms,
+               "what": "per step: the step's queries H2D from page-locked memory, kvc_decode_attention over all "
+                       "layers, outputs D2H"}
+    # the library's split rule: a merge kernel runs when a call splits the rows
+    base = w.num_layers * w.num_requests * w.num_kv_heads
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    np_max = (int(lengths.max()) + 15) // 16
+    nsplit = max(1, min(-(-4 * sms // base), 16 // w.num_layers, -(-np_max // 8))) if np_max else 1
+    if nsplit > 1:
+        pps = ((-(-np_max // nsplit)) + 3) & ~3
+        nsplit = max(1, -(-np_max // pps))
+    nsplit_launches = 2 if nsplit > 1 else 1
+    ctx.sync()
+    out_line = {
+        "metric": ATTN_METRIC, "value": value, "unit": "head-positions/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 K/V and queries)" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1) K/V with 4 outlier channels x8; N(0,1) queries)",
+        "config": {"workload": w.name + "/decode_attention", "requests_per_gpu": w.num_requests,
+                   "layers": w.num_layers, "kv_heads": w.num_kv_heads, "q_heads": w.num_q_heads,
+                   "head_dim": w.head_dim, "cache_dtype": w.dtype, "rows_per_segment": int(lengths.max()),
+                   "parallelism": f"replicas x{world} (no collective on the data path)",
+                   "l2": "inputs larger than L2: every step reads all K and V rows (tens of GB)"},
+        "roofline": roof, "e2e": e2e, "gpu_launches": args.steps * nsplit_launches, "clocks": clocks,
+    }
+    return out_line, w, lengths
+
+
+def oracle_attention_rate(w, lengths, budget_s: float):
+    """The oracle's decode attention on whole (layer, request) units until
+    ~budget_s of oracle time; head-positions/s."""
+    import numpy as np
+
+    import oracle
+    rng = np.random.default_rng(4321)
+    d, H, Hq = w.head_dim, w.num_kv_heads, w.num_q_heads
+    t_total, hp, n = 0.0, 0, 0
+    while t_total < budget_s:
+        L = int(lengths[int(rng.integers(len(lengths)))])
+        k = rng.standard_normal((H, L, d))
+        v = rng.standard_normal((H, L, d))
+        q = rng.standard_normal((Hq, d))
+        t0 = time.perf_counter()
+        oracle.decode_attention_gqa(q, k, v)
+        t_total += time.perf_counter() - t0
+        hp += L * H
+        n += 1
+    return hp / t_total, (f"{n} (layer, request) units of the workload's shape ({H} KV heads, {Hq} query heads, "
+                          f"rows = the post-round lengths), oracle float64, one thread, {t_total:.1f} s")
 
 
 # ------------------------------------------------------- oracle timing ---
@@ -448,6 +611,28 @@ def oracle_sample_rate(w, sel, budget_s: float, rank_seed: int = 0):
 
 def run_reference(args, rank, world):
     """The reference arm: the CPU oracle as it stands, on the host cores."""
+    if args.phase == "attention":
+        import numpy as np
+        w = attention_workload(args)
+        lengths = np.where(w.length <= w.budget, w.length, np.maximum(w.prompt, w.budget))
+        per_step = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+        oracle_attention_rate(w, lengths, per_step / 4 * args.warmup)
+        rates, desc = [], ""
+        for _ in range(args.steps):
+            rate, desc = oracle_attention_rate(w, lengths, per_step)
+            rates.append(rate)
+        value = statistics.mean(rates)
+        positions = int(lengths.sum()) * w.num_layers * w.num_kv_heads
+        return {
+            "impl": "reference", "metric": ATTN_METRIC, "value": value, "unit": "head-positions/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": positions / value * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name + "/decode_attention"},
+            "cpu_baseline": {"value": value, "unit": "head-positions/s", "cores": 1, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "head-positions/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
     w, sel = make_workload(args)
     per_step = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
@@ -486,6 +671,15 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
     try:
+        if args.phase == "attention":
+            out, w, lengths = run_attention(args, rank, world, dist)
+            if rank == 0:
+                if not args.no_cpu_baseline:
+                    rate, desc = oracle_attention_rate(w, lengths, 12.0)
+                    out["cpu_baseline"] = {"value": rate, "unit": "head-positions/s", "cores": 1, "kind": "oracle",
+                                           "sample": desc}
+                print(json.dumps(out), flush=True)
+            return
         out, w, sel = run_ours(args, rank, world, dist)
         if rank == 0:
             if not args.no_cpu_baseline:

@@ -49,6 +49,10 @@ KVC_SEL_BEACON = 2
 KVC_OPT_BEACON_SCORE_IMPL = 0
 KVC_OPT_BEACON_UPDATE_IMPL = 1
 
+KVC_COMPACT_ORDERED = 0
+KVC_COMPACT_HOLE_FILL = 1
+COMPACTIONS = {"ordered": KVC_COMPACT_ORDERED, "hole_fill": KVC_COMPACT_HOLE_FILL}
+
 SELECTORS = {"random": KVC_SEL_RANDOM, "random_shared": KVC_SEL_RANDOM_SHARED,
              "beacon": KVC_SEL_BEACON}
 
@@ -76,6 +80,11 @@ class kvc_round_stats(ctypes.Structure):
         return {f: getattr(self, f) for f, _ in self._fields_ if f != "reserved"}
 
 
+class kvc_round_options(ctypes.Structure):
+    _fields_ = [("sink_tokens", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("compaction", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
 class kvc_view(ctypes.Structure):
     _fields_ = [("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p),
                 ("block_table", ctypes.c_void_p), ("lengths", ctypes.c_void_p),
@@ -97,6 +106,9 @@ _SIGS = {
     "kvc_append": (_i32, [_P, _P, _i32, _i32, _P, _P, _P, _i32]),
     "kvc_update_beacons": (_i32, [_P, _P, _P]),
     "kvc_compress": (_i32, [_P, _i32, _P, _u64, _P, ctypes.POINTER(kvc_round_stats)]),
+    "kvc_compress_ex": (_i32, [_P, _i32, _P, _u64, ctypes.POINTER(kvc_round_options), _P,
+                               ctypes.POINTER(kvc_round_stats)]),
+    "kvc_decode_attention": (_i32, [_P, _i32, _i32, _P, ctypes.c_float, _P, _P, _P]),
     "kvc_gather_view": (_i32, [_P, ctypes.POINTER(kvc_view)]),
     "kvc_get_lengths": (_i32, [_P, _P, _P]),
     "kvc_gather_dense": (_i32, [_P, _i32, _i32, _i32, _i32, _P, _P, _P]),
@@ -220,15 +232,42 @@ class Context:
                self.handle)
         return ms.value if timed else None
 
-    def compress(self, selector, budgets, seed: int, debug_scores=None, stats: bool = False):
+    def compress(self, selector, budgets, seed: int, debug_scores=None, stats: bool = False,
+                 sink_tokens=None, block: int = 1, compaction="ordered"):
+        """One eviction round (kvc_compress_ex).  sink_tokens None protects the
+        whole prompt; block and compaction as in kvc_round_options."""
         sel = SELECTORS[selector] if isinstance(selector, str) else int(selector)
         b = np.ascontiguousarray(budgets, dtype=np.int32)
         if b.shape != (self.spec.num_requests,):
             raise ValueError("budgets must have one entry per request")
+        comp = COMPACTIONS[compaction] if isinstance(compaction, str) else int(compaction)
+        opts = kvc_round_options(-1 if sink_tokens is None else int(sink_tokens), int(block), comp, 0)
         st = kvc_round_stats()
-        _check(kvc_compress(self.handle, sel, b.ctypes.data_as(_P), ctypes.c_uint64(seed),
-                            _ptr(debug_scores), ctypes.byref(st) if stats else None), self.handle)
+        _check(kvc_compress_ex(self.handle, sel, b.ctypes.data_as(_P), ctypes.c_uint64(seed),
+                               ctypes.byref(opts), _ptr(debug_scores),
+                               ctypes.byref(st) if stats else None), self.handle)
         return st.as_dict() if stats else None
+
+    def decode_attention(self, q, layer_begin: int = 0, out=None, lse=None, scale: float = 0.0,
+                         with_lse: bool = True, timed: bool = False):
+        """kvc_decode_attention for q [layer_count, R, Hq, d] (cache dtype, on the
+        context's device).  Returns (out, lse) float32 tensors, plus the device
+        time in ms when timed."""
+        import torch
+        s = self.spec
+        if q.dim() != 4 or q.shape[1:] != (s.num_requests, s.num_q_heads, s.head_dim) or q.dtype != self.dtype:
+            raise ValueError("q must be [layer_count, num_requests, num_q_heads, head_dim] in the cache dtype")
+        q = q.contiguous()
+        lc = q.shape[0]
+        if out is None:
+            out = torch.empty((lc, s.num_requests, s.num_q_heads, s.head_dim), dtype=torch.float32,
+                              device=self.device)
+        if lse is None and with_lse:
+            lse = torch.empty((lc, s.num_requests, s.num_q_heads), dtype=torch.float32, device=self.device)
+        ms = ctypes.c_float(0.0)
+        _check(kvc_decode_attention(self.handle, int(layer_begin), int(lc), _ptr(q), ctypes.c_float(scale),
+                                    _ptr(out), _ptr(lse), ctypes.byref(ms) if timed else None), self.handle)
+        return (out, lse, ms.value) if timed else (out, lse)
 
     def sync(self):
         _check(kvc_sync(self.handle), self.handle)

@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -29,8 +30,11 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
   size_t bt, len, prompt, pos, qring, beacons, beacons_s, counts, scores, lse, status, counters,
-      stage, total, stage_slot;
+      stage, attn, total, stage_slot;
 };
+
+// Split partials of the decode attention: room for this many splits of one layer.
+constexpr int kAttnSplits = 16;
 
 int elem_size(int dtype) { return dtype == KVC_BF16 ? 2 : 4; }
 
@@ -86,6 +90,7 @@ Layout make_layout(const kvc_config &c) {
   L.counters = take(256);
   L.stage_slot = align_up(R * 16 + R * maxp * 8 + R * 8 + 1024, 256);
   L.stage = take(L.stage_slot * kStageSlots);
+  L.attn = take(R * Hq * (d + 2) * 4 * (size_t)kAttnSplits);
   L.total = off;
   return L;
 }
@@ -115,11 +120,13 @@ struct kvc_ctx {
   std::vector<int32_t> h_bt, h_len, h_prompt;
   std::vector<int64_t> h_next_pos, q_total, q_last;
   std::vector<uint8_t> h_binit;
+  std::vector<uint8_t> h_unordered;  // a hole-filling round left slots out of position order
   std::vector<int32_t> free_pages;
   int64_t round = 0;
   int score_impl = 0;
   int update_impl = 0;
-  int es = 2, row_bytes = 0, G = 1, maxp = 0;
+  int es = 2, row_bytes = 0, G = 1, maxp = 0, num_sms = 148;
+  float *d_attn = nullptr;
   std::string err;
 };
 
@@ -289,6 +296,11 @@ kvc_status kvc_create(const kvc_config *cfg, void *k_pool, void *v_pool, void *w
   c->d_status = reinterpret_cast<int32_t *>(c->ws + lay.status);
   c->d_counters = reinterpret_cast<unsigned long long *>(c->ws + lay.counters);
   c->d_stage = c->ws + lay.stage;
+  c->d_attn = reinterpret_cast<float *>(c->ws + lay.attn);
+  if (cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    c->num_sms = 148;
+  }
   const int R = cfg->num_requests;
   c->h_bt.assign((size_t)R * c->maxp, -1);
   c->h_len.assign(R, 0);
@@ -297,6 +309,7 @@ kvc_status kvc_create(const kvc_config *cfg, void *k_pool, void *v_pool, void *w
   c->q_total.assign(R, 0);
   c->q_last.assign(R, 0);
   c->h_binit.assign(R, 0);
+  c->h_unordered.assign(R, 0);
   c->free_pages.resize((size_t)cfg->num_pages);
   for (int64_t i = 0; i < cfg->num_pages; ++i)
     c->free_pages[(size_t)i] = (int32_t)(cfg->num_pages - 1 - i);  // pop_back gives 0, 1, ...
@@ -531,11 +544,25 @@ kvc_status kvc_update_beacons(kvc_ctx *ctx, int32_t *assign_out, float *ms_out) 
 
 kvc_status kvc_compress(kvc_ctx *ctx, kvc_selector selector, const int32_t *budgets,
                         uint64_t seed, void *debug_scores, kvc_round_stats *stats) {
+  return kvc_compress_ex(ctx, selector, budgets, seed, nullptr, debug_scores, stats);
+}
+
+kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *budgets,
+                           uint64_t seed, const kvc_round_options *opts, void *debug_scores,
+                           kvc_round_stats *stats) {
   if (!ctx) return KVC_ERR_INVALID_ARG;
   const kvc_config &c = ctx->cfg;
   if (selector != KVC_SEL_RANDOM && selector != KVC_SEL_RANDOM_SHARED && selector != KVC_SEL_BEACON)
     return fail(ctx, KVC_ERR_INVALID_ARG, "unknown selector");
   if (!budgets) return fail(ctx, KVC_ERR_INVALID_ARG, "budgets is NULL");
+  const kvc_round_options o = opts ? *opts : kvc_round_options{-1, 1, KVC_COMPACT_ORDERED, 0};
+  if (o.block < 1 || o.block > kMaxSeqLen)
+    return fail(ctx, KVC_ERR_INVALID_ARG, "block must be in [1, 32768]");
+  if (o.block != 1 && selector == KVC_SEL_BEACON)
+    return fail(ctx, KVC_ERR_INVALID_ARG, "block-granular draws apply to the random selectors only");
+  if (o.compaction != KVC_COMPACT_ORDERED && o.compaction != KVC_COMPACT_HOLE_FILL)
+    return fail(ctx, KVC_ERR_INVALID_ARG, "unknown compaction");
+  if (o.reserved != 0) return fail(ctx, KVC_ERR_INVALID_ARG, "reserved option field must be 0");
   KVC_CUDA(ctx, cudaSetDevice(ctx->device));
   if (debug_scores && !device_ptr_on(ctx->device, debug_scores))
     return fail(ctx, KVC_ERR_INVALID_ARG, "debug_scores must be device memory");
@@ -546,11 +573,13 @@ kvc_status kvc_compress(kvc_ctx *ctx, kvc_selector selector, const int32_t *budg
   st.round = ctx->round;
   st.segments = (int64_t)R * per_req_segs;
   std::vector<SegDesc> segs;
-  std::vector<int32_t> new_len(ctx->h_len);
+  std::vector<int32_t> new_len(ctx->h_len), new_prompt(ctx->h_prompt);
+  bool tie_by_pos = false;
   for (int r = 0; r < R; ++r) {
     const int K = budgets[r];
     if (K < 0) return fail(ctx, KVC_ERR_INVALID_ARG, "negative budget for request " + std::to_string(r));
-    const int L = ctx->h_len[r], P = ctx->h_prompt[r];
+    const int L = ctx->h_len[r];
+    const int P = o.sink_tokens < 0 ? ctx->h_prompt[r] : std::min(ctx->h_prompt[r], o.sink_tokens);
     st.head_positions += (int64_t)L * per_req_segs;
     if (L <= K) {
       st.noop_segments += per_req_segs;
@@ -561,10 +590,12 @@ kvc_status kvc_compress(kvc_ctx *ctx, kvc_selector selector, const int32_t *budg
     st.candidates += (int64_t)(L - P) * per_req_segs;
     st.evicted += (int64_t)(L - P - M) * per_req_segs;
     new_len[r] = P + M;
+    new_prompt[r] = P;
     if (M > 0) {
       if (selector == KVC_SEL_BEACON && !ctx->h_binit[r])
         return fail(ctx, KVC_ERR_STATE, "request " + std::to_string(r) + " has no beacons yet (call kvc_update_beacons)");
       segs.push_back(SegDesc{r, L, P, M});
+      tie_by_pos = tie_by_pos || ctx->h_unordered[r];
     }
   }
   if (selector == KVC_SEL_BEACON && c.num_beacons == 0)
@@ -578,7 +609,8 @@ kvc_status kvc_compress(kvc_ctx *ctx, kvc_selector selector, const int32_t *budg
   if (kvc_status s = stage_acquire(ctx, sd_stage)) return s;
   std::memcpy(sd_stage.h, segs.data(), seg_bytes);
   std::memcpy(sd_stage.h + align_up(seg_bytes, 16), new_len.data(), (size_t)R * 4);
-  if (kvc_status s = stage_upload(ctx, sd_stage, align_up(seg_bytes, 16) + (size_t)R * 4)) return s;
+  std::memcpy(sd_stage.h + align_up(seg_bytes, 16) + (size_t)R * 4, new_prompt.data(), (size_t)R * 4);
+  if (kvc_status s = stage_upload(ctx, sd_stage, align_up(seg_bytes, 16) + (size_t)R * 8)) return s;
   const SegDesc *d_segs = reinterpret_cast<const SegDesc *>(sd_stage.d);
   const bool timed = stats != nullptr;
   if (timed) {
@@ -631,6 +663,8 @@ kvc_status kvc_compress(kvc_ctx *ctx, kvc_selector selector, const int32_t *budg
   sp.hkv = c.num_kv_heads;
   sp.row_bytes = ctx->row_bytes;
   sp.max_seq = c.max_seq_len;
+  sp.block = o.block;
+  sp.flags = (o.compaction == KVC_COMPACT_HOLE_FILL ? kScHoleFill : 0) | (tie_by_pos ? kScTieByPos : 0);
   sp.seed = seed;
   sp.round = (uint64_t)ctx->round;
   const int mode = selector == KVC_SEL_RANDOM ? kModeRandom
@@ -656,6 +690,9 @@ kvc_status kvc_compress(kvc_ctx *ctx, kvc_selector selector, const int32_t *budg
   if (timed) KVC_CUDA(ctx, cudaEventRecord(ctx->ev[2], ctx->stream));
   KVC_CUDA(ctx, cudaMemcpyAsync(ctx->d_len, sd_stage.d + align_up(seg_bytes, 16), (size_t)R * 4,
                                 cudaMemcpyDeviceToDevice, ctx->stream));
+  if (new_prompt != ctx->h_prompt)
+    KVC_CUDA(ctx, cudaMemcpyAsync(ctx->d_prompt, sd_stage.d + align_up(seg_bytes, 16) + (size_t)R * 4,
+                                  (size_t)R * 4, cudaMemcpyDeviceToDevice, ctx->stream));
   if (kvc_status s = stage_release(ctx, sd_stage)) return s;
   // host mirror: lengths and freed pages
   for (int r = 0; r < R; ++r) {
@@ -668,6 +705,9 @@ kvc_status kvc_compress(kvc_ctx *ctx, kvc_selector selector, const int32_t *budg
     }
     ctx->h_len[r] = Rn;
   }
+  ctx->h_prompt = new_prompt;
+  if (o.compaction == KVC_COMPACT_HOLE_FILL)
+    for (const auto &sg : segs) ctx->h_unordered[sg.req] = 1;
   ctx->round += 1;
   if (timed) {
     KVC_CUDA(ctx, cudaStreamSynchronize(ctx->stream));
@@ -730,6 +770,74 @@ kvc_status kvc_gather_dense(kvc_ctx *ctx, int32_t layer, int32_t req_begin, int3
                                       c.num_pages, ctx->maxp, static_cast<uint8_t *>(k_out),
                                       static_cast<uint8_t *>(v_out), pos_out, ctx->stream);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "gather_dense");
+  return KVC_OK;
+}
+
+kvc_status kvc_decode_attention(kvc_ctx *ctx, int32_t layer_begin, int32_t layer_count, const void *q,
+                                float scale, float *out, float *lse, float *ms_out) {
+  if (!ctx) return KVC_ERR_INVALID_ARG;
+  const kvc_config &c = ctx->cfg;
+  if (layer_begin < 0 || layer_count < 1 || layer_begin + layer_count > c.num_layers)
+    return fail(ctx, KVC_ERR_INVALID_ARG, "layer range out of bounds");
+  if (!q || !out) return fail(ctx, KVC_ERR_INVALID_ARG, "q and out are required");
+  if (!(scale >= 0.f) || !std::isfinite(scale)) return fail(ctx, KVC_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  KVC_CUDA(ctx, cudaSetDevice(ctx->device));
+  if (!device_ptr_on(ctx->device, q) || !device_ptr_on(ctx->device, out) ||
+      (lse && !device_ptr_on(ctx->device, lse)))
+    return fail(ctx, KVC_ERR_INVALID_ARG, "q, out and lse must be device memory of the context's device");
+  if (((uintptr_t)q % ctx->es) || ((uintptr_t)out & 3) || ((uintptr_t)lse & 3))
+    return fail(ctx, KVC_ERR_INVALID_ARG, "q, out or lse misaligned");
+  const int G = ctx->G;
+  const int64_t pool_rows = (int64_t)c.num_layers * c.num_pages * c.num_kv_heads * kPage;
+  if (!decode_attention_supported(c.dtype, c.head_dim, G) || pool_rows >= ((int64_t)1 << 31))
+    return fail(ctx, KVC_ERR_UNSUPPORTED,
+                "decode attention needs bf16 or f32, head_dim 64 or 128, 1, 2, 4 or 8 query heads per KV "
+                "head and fewer than 2^31 pool rows");
+  const int R = c.num_requests;
+  int max_len = 0;
+  for (int r = 0; r < R; ++r) max_len = std::max(max_len, ctx->h_len[r]);
+  const int np_max = (max_len + kPage - 1) / kPage;
+  // splits: enough CTAs for two waves of two CTAs per SM, pages of a split a
+  // multiple of the 4-page tile, at least two tiles per split
+  const int64_t base = (int64_t)layer_count * R * c.num_kv_heads;
+  int nsplit = 1;
+  if (np_max > 0) {
+    const int64_t want = (4LL * ctx->num_sms + base - 1) / base;
+    nsplit = (int)std::max<int64_t>(1, std::min<int64_t>({want, kAttnSplits / layer_count, (np_max + 7) / 8}));
+  }
+  int pps = std::max(1, (np_max + nsplit - 1) / nsplit);
+  pps = (pps + 3) & ~3;
+  nsplit = std::max(1, (np_max + pps - 1) / pps);
+  DecodeAttnParams p{};
+  p.q = static_cast<const uint8_t *>(q);
+  p.block_table = ctx->d_bt;
+  p.lengths = ctx->d_len;
+  p.out = out;
+  p.lse = lse;
+  p.part_o = ctx->d_attn;
+  p.part_ml = ctx->d_attn + (size_t)layer_count * R * c.num_q_heads * nsplit * c.head_dim;
+  p.status = ctx->d_status;
+  p.num_pages = c.num_pages;
+  p.bt_stride = ctx->maxp;
+  p.layer_begin = layer_begin;
+  p.layer_count = layer_count;
+  p.R = R;
+  p.hkv = c.num_kv_heads;
+  p.hq = c.num_q_heads;
+  p.nsplit = nsplit;
+  p.pages_per_split = pps;
+  p.qscale = (scale > 0.f ? scale : 1.0f / std::sqrt((float)c.head_dim)) * 1.4426950408889634f;
+  if (ms_out) KVC_CUDA(ctx, cudaEventRecord(ctx->ev[0], ctx->stream));
+  int launches = 0;
+  cudaError_t e = launch_decode_attention(p, ctx->k_pool, ctx->v_pool, pool_rows, c.head_dim, c.dtype, G,
+                                          &launches, ctx->stream);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "decode_attention");
+  if (ms_out) {
+    KVC_CUDA(ctx, cudaEventRecord(ctx->ev[1], ctx->stream));
+    KVC_CUDA(ctx, cudaEventSynchronize(ctx->ev[1]));
+    KVC_CUDA(ctx, cudaEventElapsedTime(ms_out, ctx->ev[0], ctx->ev[1]));
+    return take_device_status(ctx);
+  }
   return KVC_OK;
 }
 

@@ -41,7 +41,28 @@ struct SelectCompactParams {
   int32_t *status;
   int64_t num_pages;
   int32_t bt_stride, layers, hkv, row_bytes, max_seq;
+  int32_t block;  // positions per Philox draw (random selectors)
+  int32_t flags;  // kScTieByPos | kScHoleFill
   uint64_t seed, round;
+};
+
+// SelectCompactParams::flags
+constexpr int kScTieByPos = 1;  // slots may be out of position order: split ties by position
+constexpr int kScHoleFill = 2;  // hole-filling compaction (implies ties by position)
+
+// One decode step of attention over the cache (decode_attention.cu).
+struct DecodeAttnParams {
+  const uint8_t *q;            // [layer_count][R][Hq][d] dtype
+  const int32_t *block_table;  // [R][bt_stride]
+  const int32_t *lengths;      // [R] device lengths
+  float *out;                  // [layer_count][R][Hq][d]
+  float *lse;                  // [layer_count][R][Hq] or null
+  float *part_o;               // split partials [layer_count][R][Hq][nsplit][d]
+  float *part_ml;              // [layer_count][R][Hq][nsplit][2] (max in base 2, sum)
+  int32_t *status;
+  int64_t num_pages;
+  int32_t bt_stride, layer_begin, layer_count, R, hkv, hq, nsplit, pages_per_split;
+  float qscale;                // scale * log2(e)
 };
 
 // Beacon update over the query ring.
@@ -90,6 +111,10 @@ cudaError_t launch_gather_dense(const uint8_t *k_pool, const uint8_t *v_pool,
                                 const int32_t *lengths, int layer, int req_begin, int req_count,
                                 int cap, int hkv, int row_bytes, int64_t num_pages, int bt_stride,
                                 uint8_t *k_out, uint8_t *v_out, int32_t *pos_out, cudaStream_t s);
+bool decode_attention_supported(int dtype, int head_dim, int G);
+cudaError_t launch_decode_attention(const DecodeAttnParams &p, const void *k_pool, const void *v_pool,
+                                    int64_t pool_rows, int head_dim, int dtype, int G, int *launches,
+                                    cudaStream_t s);
 cudaError_t launch_select_compact(const SelectCompactParams &p, int mode, int n_seg_req,
                                   int max_n, int max_m, cudaStream_t s);
 cudaError_t launch_beacon_update(const BeaconUpdateParams &p, int n_req, cudaStream_t s);

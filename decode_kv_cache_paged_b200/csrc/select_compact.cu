@@ -3,31 +3,37 @@
 // survivors in place.
 //
 // What it computes (Random Attention article, "Random Attention：不判断重要性，
-// 只随机保留" and "发现四"): the prompt slots [0, P) are never candidates; the
-// N = L - P generated slots are ranked by (score desc, original position asc),
-// the best M stay and are packed, in their original order, into slots P,
-// P+1, ...; K rows, V rows and the position map move together.  The score is
-// the Philox draw of the (position, head, layer, request) counter for the
-// random selectors, or the precomputed beacon score.
+// 只随机保留" and "发现四"): the protected slots [0, P) are never candidates;
+// the N = L - P candidate slots are ranked by (score desc, original position
+// asc), the best M stay and are compacted into slots [P, P + M); K rows, V
+// rows and the position map move together.  The score is the Philox draw of
+// the (position / block, head, layer, request) counter for the random
+// selectors (block = 1: one draw per position; larger blocks keep contiguous
+// runs, "发现二"), or the precomputed beacon score.
 //
 // Design (B200): one CTA per segment, everything between score and copy in
 // shared memory.
 //   1. score: each thread draws the 32-bit keys of a strided set of slots
 //      (the random path reads only the 4-byte position map, never K/V);
 //   2. select: 4-pass MSB radix select (8-bit digits, shared-memory
-//      histogram) finds the M-th largest key tau and how many keys equal to
-//      tau stay (the lowest slots among them, which hold the lowest
-//      positions because slots are kept in position order);
-//   3. ranks: tile-wise block scan of (key > tau, key == tau) with warp
-//      ballots gives every survivor its destination rank; the inverse map
-//      rank -> source slot is kept as uint16 in shared memory;
-//   4. copy: survivors from the first evicted slot on move to slot P + rank.
-//      Each chunk of ranks (8 rows per thread group, 64-128 KB of K and V in
-//      flight per CTA) is read (16-byte vector loads, K and V rows plus
-//      the position entry) into registers, the CTA synchronises, then writes.
-//      A chunk only writes slots below its own highest source slot, and the
-//      next chunk only reads slots above it, so one barrier per chunk makes
-//      the in-place move safe while loads of chunk c+1 overlap stores of c.
+//      histogram) finds the M-th largest key tau, how many keys equal tau and
+//      how many of those stay.  When slots are in position order (always, as
+//      long as no round filled holes) the tied keys that stay are the lowest
+//      slots; otherwise a second radix select over the tied candidates on the
+//      complemented position picks the lowest positions exactly;
+//   3. ranks: tile-wise block scans with warp ballots give every survivor
+//      its rank (order-preserving compaction) or list the holes and the
+//      survivors past the new length (hole filling);
+//   4. copy, order-preserving: survivors from the first evicted slot on move
+//      to slot P + rank.  Each chunk of ranks (8 rows per thread group,
+//      64-128 KB of K and V in flight per CTA) is read with 16-byte vector
+//      loads into registers, the CTA synchronises, then writes.  A chunk only
+//      writes slots below its own highest source slot and the next chunk only
+//      reads slots above it, so one barrier per chunk makes the in-place move
+//      safe while loads of chunk c+1 overlap stores of chunk c;
+//   4'. copy, hole filling: the i-th survivor at or past the new length moves
+//      into the i-th evicted slot below it; sources and destinations are
+//      disjoint, so the copies need no barrier.
 // Rows of the same segment are never touched by another CTA.
 #include "kvc_internal.h"
 #include "philox.cuh"
@@ -42,17 +48,23 @@ namespace {
 #define KVC_SC_UNROLL_LARGE 8
 #endif
 
+// copy / tie variants of the kernel
+constexpr int kOrderedSlotTie = 0;  // order-preserving, ties by slot (slots in position order)
+constexpr int kOrderedPosTie = 1;   // order-preserving, ties by position
+constexpr int kHoleFill = 2;        // hole filling, ties by position
+
 __device__ __forceinline__ uint32_t float_order_key(float f) {
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-template <int NT>
-__device__ __forceinline__ void block_radix_select(const uint32_t *keys, int n, int k_in,
-                                                   uint32_t *hist, uint32_t *bcast,
-                                                   uint32_t &tau, int &need) {
-  // Finds the k_in-th largest key (1-based) and how many keys equal to it
-  // belong to the top k_in.
+// k_in-th largest key (1-based) among the candidates for which keyfn(j, key)
+// returns true; also how many keys equal it (count_eq) and how many of those
+// belong to the top k_in (need).
+template <int NT, class KeyFn>
+__device__ __forceinline__ void block_radix_select(int n, int k_in, KeyFn keyfn, uint32_t *hist,
+                                                   uint32_t *bcast, uint32_t &tau, int &need,
+                                                   int &count_eq) {
   uint32_t prefix = 0, mask = 0;
   int k = k_in;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -61,8 +73,8 @@ __device__ __forceinline__ void block_radix_select(const uint32_t *keys, int n, 
     for (int i = tid; i < 256; i += NT) hist[i] = 0;
     __syncthreads();
     for (int j = tid; j < n; j += NT) {
-      const uint32_t key = keys[j];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      uint32_t key;
+      if (keyfn(j, key) && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
     if (warp == 0) {
@@ -86,36 +98,68 @@ __device__ __forceinline__ void block_radix_select(const uint32_t *keys, int n, 
       if (lane == first) {
         uint32_t cum = excl;
         int digit = 0;
+        uint32_t cnt = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           if (cum + c[i] >= (uint32_t)k) {
             digit = 255 - 8 * lane - i;
+            cnt = c[i];
             break;
           }
           cum += c[i];
         }
         bcast[0] = (uint32_t)digit;
         bcast[1] = (uint32_t)k - cum;
+        bcast[2] = cnt;
       }
     }
     __syncthreads();
     prefix |= bcast[0] << shift;
     mask |= 255u << shift;
     k = (int)bcast[1];
+    count_eq = (int)bcast[2];
     __syncthreads();
   }
   tau = prefix;
   need = k;
 }
 
-template <int NT, int MODE, int kUnroll>
+// Tile-wise exclusive scan of a per-candidate predicate over [lo, hi) in
+// candidate order; calls fn(j, index) for every j with pred(j) true, index =
+// number of earlier candidates with pred true.  Returns the total.
+template <int NT, class Pred, class Fn>
+__device__ __forceinline__ int block_scan_each(int lo, int hi, Pred pred, Fn fn, uint32_t *warp_cnt) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int carry = 0;
+#pragma unroll 1
+  for (int base = lo; base < hi; base += NT) {
+    const int j = base + tid;
+    const bool f = j < hi && pred(j);
+    const unsigned m = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) warp_cnt[warp] = __popc(m);
+    __syncthreads();
+    int off = carry, tot = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+      const int c = warp_cnt[w];
+      if (w < warp) off += c;
+      tot += c;
+    }
+    if (f) fn(j, off + __popc(m & ((1u << lane) - 1u)));
+    carry += tot;
+    __syncthreads();  // warp_cnt reuse
+  }
+  return carry;
+}
+
+template <int NT, int MODE, int kUnroll, int VAR>
 __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams p, int keys_cap) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint32_t *keys = reinterpret_cast<uint32_t *>(smem);                  // [keys_cap]
   uint16_t *src_of_rank = reinterpret_cast<uint16_t *>(keys + keys_cap);  // [keys_cap]
   __shared__ uint32_t hist[256];
-  __shared__ uint32_t bcast[2];
-  __shared__ uint32_t warp_gt[NT / 32], warp_eq[NT / 32];
+  __shared__ uint32_t bcast[3];
+  __shared__ uint32_t warp_cnt[NT / 32], warp_eq[NT / 32];
   __shared__ int first_evicted;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -141,7 +185,7 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
       key = float_order_key(p.scores[seg_flat * p.max_seq + j]);
     } else {
       const int pos = p.pos_map[row_of(P + j)];
-      key = philox4x64_10_word0_hi32((uint64_t)(int64_t)pos, head_field, (uint64_t)l,
+      key = philox4x64_10_word0_hi32((uint64_t)(int64_t)(pos / p.block), head_field, (uint64_t)l,
                                      (uint64_t)r, p.seed, p.round);
       if (p.debug) p.debug[seg_flat * p.max_seq + j] = key;
     }
@@ -151,118 +195,192 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
 
   // 2. threshold
   uint32_t tau;
-  int need;
-  block_radix_select<NT>(keys, N, M, hist, bcast, tau, need);
-
-  // 3. ranks (tiles of NT slots in slot order)
-  int carry_gt = 0, carry_eq = 0;
-#pragma unroll 1
-  for (int base = 0; base < N; base += NT) {
-    const int j = base + tid;
-    const bool valid = j < N;
-    const uint32_t key = valid ? keys[j] : 0u;
-    const bool gt = valid && key > tau;
-    const bool eq = valid && key == tau;
-    const unsigned mgt = __ballot_sync(0xffffffffu, gt);
-    const unsigned meq = __ballot_sync(0xffffffffu, eq);
-    const unsigned lt_mask = (1u << lane) - 1u;
-    if (lane == 0) {
-      warp_gt[warp] = __popc(mgt);
-      warp_eq[warp] = __popc(meq);
-    }
-    __syncthreads();
-    int off_gt = carry_gt, off_eq = carry_eq, tot_gt = 0, tot_eq = 0;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w) {
-      const int g = warp_gt[w], e = warp_eq[w];
-      if (w < warp) {
-        off_gt += g;
-        off_eq += e;
-      }
-      tot_gt += g;
-      tot_eq += e;
-    }
-    const int gt_before = off_gt + __popc(mgt & lt_mask);
-    const int eq_before = off_eq + __popc(meq & lt_mask);
-    const bool kept = gt || (eq && eq_before < need);
-    if (kept) {
-      const int rank = gt_before + min(eq_before, need);
-      src_of_rank[rank] = (uint16_t)j;
-    } else if (valid) {
-      atomicMin(&first_evicted, j);
-    }
-    carry_gt += tot_gt;
-    carry_eq += tot_eq;
-    __syncthreads();  // warp_gt/warp_eq reuse
+  int need, count_eq;
+  block_radix_select<NT>(
+      N, M, [&](int j, uint32_t &k) { k = keys[j]; return true; }, hist, bcast, tau, need, count_eq);
+  // with ties split and slots possibly out of position order: the `need`
+  // lowest positions among the tied keys (positions are distinct)
+  uint32_t ptau = 0;
+  const bool split_by_pos = VAR != kOrderedSlotTie && need < count_eq;
+  if (split_by_pos) {
+    int need2, cnt2;
+    block_radix_select<NT>(
+        N, need,
+        [&](int j, uint32_t &k) {
+          if (keys[j] != tau) return false;
+          k = ~(uint32_t)p.pos_map[row_of(P + j)];
+          return true;
+        },
+        hist, bcast, ptau, need2, cnt2);
   }
-  __syncthreads();
+  auto kept_pos = [&](int j) -> bool {  // kept flag when ties go by position
+    const uint32_t key = keys[j];
+    if (key != tau) return key > tau;
+    if (!split_by_pos) return true;
+    return ~(uint32_t)p.pos_map[row_of(P + j)] >= ptau;
+  };
 
-  // 4. in-place, order-preserving copy of ranks [first_evicted, M)
-  const int q0 = first_evicted;
   const int vpr = p.row_bytes >> 4;  // 16-byte vectors per row
   const int rows_per_pass = NT / vpr;
   const int my_row = tid / vpr, my_vec = tid - (tid / vpr) * vpr;
   const bool active = my_row < rows_per_pass;
   const int64_t rb = p.row_bytes;
+
+  if (VAR != kHoleFill) {
+    // 3. ranks in slot order
+    if (VAR == kOrderedSlotTie) {
+      // kept = key > tau, or key == tau among the first `need` such slots
+      int carry_gt = 0, carry_eq = 0;
 #pragma unroll 1
-  for (int base = q0; base < M; base += rows_per_pass * kUnroll) {
-    uint4 kr[kUnroll], vr[kUnroll];
-    int pr[kUnroll];
-    int64_t drow[kUnroll];
+      for (int base = 0; base < N; base += NT) {
+        const int j = base + tid;
+        const bool valid = j < N;
+        const uint32_t key = valid ? keys[j] : 0u;
+        const bool gt = valid && key > tau;
+        const bool eq = valid && key == tau;
+        const unsigned mgt = __ballot_sync(0xffffffffu, gt);
+        const unsigned meq = __ballot_sync(0xffffffffu, eq);
+        const unsigned lt_mask = (1u << lane) - 1u;
+        if (lane == 0) {
+          warp_cnt[warp] = __popc(mgt);
+          warp_eq[warp] = __popc(meq);
+        }
+        __syncthreads();
+        int off_gt = carry_gt, off_eq = carry_eq, tot_gt = 0, tot_eq = 0;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int q = base + u * rows_per_pass + my_row;
-      drow[u] = -1;
-      if (active && q < M) {
-        const int64_t srow = row_of(P + src_of_rank[q]);
-        drow[u] = row_of(P + q);
-        kr[u] = *reinterpret_cast<const uint4 *>(p.k_pool + srow * rb + my_vec * 16);
-        vr[u] = *reinterpret_cast<const uint4 *>(p.v_pool + srow * rb + my_vec * 16);
-        if (my_vec == 0) pr[u] = p.pos_map[srow];
+        for (int w = 0; w < NT / 32; ++w) {
+          const int g = warp_cnt[w], e = warp_eq[w];
+          if (w < warp) {
+            off_gt += g;
+            off_eq += e;
+          }
+          tot_gt += g;
+          tot_eq += e;
+        }
+        const int gt_before = off_gt + __popc(mgt & lt_mask);
+        const int eq_before = off_eq + __popc(meq & lt_mask);
+        const bool kept = gt || (eq && eq_before < need);
+        if (kept) {
+          src_of_rank[gt_before + min(eq_before, need)] = (uint16_t)j;
+        } else if (valid) {
+          atomicMin(&first_evicted, j);
+        }
+        carry_gt += tot_gt;
+        carry_eq += tot_eq;
+        __syncthreads();
       }
+    } else {
+      block_scan_each<NT>(
+          0, N, [&](int j) { return kept_pos(j); },
+          [&](int j, int rank) { src_of_rank[rank] = (uint16_t)j; }, warp_cnt);
+      for (int j = tid; j < N; j += NT)
+        if (!kept_pos(j)) atomicMin(&first_evicted, j);
     }
     __syncthreads();
+
+    // 4. in-place, order-preserving copy of ranks [first_evicted, M)
+    const int q0 = first_evicted;
+#pragma unroll 1
+    for (int base = q0; base < M; base += rows_per_pass * kUnroll) {
+      uint4 kr[kUnroll], vr[kUnroll];
+      int pr[kUnroll];
+      int64_t drow[kUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (drow[u] >= 0) {
-        *reinterpret_cast<uint4 *>(p.k_pool + drow[u] * rb + my_vec * 16) = kr[u];
-        *reinterpret_cast<uint4 *>(p.v_pool + drow[u] * rb + my_vec * 16) = vr[u];
-        if (my_vec == 0) p.pos_map[drow[u]] = pr[u];
+      for (int u = 0; u < kUnroll; ++u) {
+        const int q = base + u * rows_per_pass + my_row;
+        drow[u] = -1;
+        if (active && q < M) {
+          const int64_t srow = row_of(P + src_of_rank[q]);
+          drow[u] = row_of(P + q);
+          kr[u] = *reinterpret_cast<const uint4 *>(p.k_pool + srow * rb + my_vec * 16);
+          vr[u] = *reinterpret_cast<const uint4 *>(p.v_pool + srow * rb + my_vec * 16);
+          if (my_vec == 0) pr[u] = p.pos_map[srow];
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (drow[u] >= 0) {
+          *reinterpret_cast<uint4 *>(p.k_pool + drow[u] * rb + my_vec * 16) = kr[u];
+          *reinterpret_cast<uint4 *>(p.v_pool + drow[u] * rb + my_vec * 16) = vr[u];
+          if (my_vec == 0) p.pos_map[drow[u]] = pr[u];
+        }
       }
     }
+    if (tid == 0 && M > q0) atomicAdd(p.counters, (unsigned long long)(M - q0));
+  } else {
+    // 3'. holes (evicted candidates below M) and movers (kept at or past M),
+    // each listed in candidate order: holes at src_of_rank[0..), movers at
+    // src_of_rank[M..)
+    const int n_holes = block_scan_each<NT>(
+        0, M, [&](int j) { return !kept_pos(j); },
+        [&](int j, int i) { src_of_rank[i] = (uint16_t)j; }, warp_cnt);
+    block_scan_each<NT>(
+        M, N, [&](int j) { return kept_pos(j); },
+        [&](int j, int i) { src_of_rank[M + i] = (uint16_t)j; }, warp_cnt);
+    __syncthreads();
+    // 4'. the i-th mover goes to the i-th hole; all copies are independent
+#pragma unroll 1
+    for (int base = 0; base < n_holes; base += rows_per_pass * kUnroll) {
+      uint4 kr[kUnroll], vr[kUnroll];
+      int pr[kUnroll];
+      int64_t drow[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int i = base + u * rows_per_pass + my_row;
+        drow[u] = -1;
+        if (active && i < n_holes) {
+          const int64_t srow = row_of(P + src_of_rank[M + i]);
+          drow[u] = row_of(P + src_of_rank[i]);
+          kr[u] = *reinterpret_cast<const uint4 *>(p.k_pool + srow * rb + my_vec * 16);
+          vr[u] = *reinterpret_cast<const uint4 *>(p.v_pool + srow * rb + my_vec * 16);
+          if (my_vec == 0) pr[u] = p.pos_map[srow];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (drow[u] >= 0) {
+          *reinterpret_cast<uint4 *>(p.k_pool + drow[u] * rb + my_vec * 16) = kr[u];
+          *reinterpret_cast<uint4 *>(p.v_pool + drow[u] * rb + my_vec * 16) = vr[u];
+          if (my_vec == 0) p.pos_map[drow[u]] = pr[u];
+        }
+      }
+    }
+    if (tid == 0 && n_holes > 0) atomicAdd(p.counters, (unsigned long long)n_holes);
   }
-  if (tid == 0 && M > q0) atomicAdd(p.counters, (unsigned long long)(M - q0));
+}
+
+template <int NT, int U, int MODE, int VAR>
+cudaError_t launch_one(const SelectCompactParams &p, int n_seg_req, int keys_cap, size_t smem,
+                       cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(select_compact_kernel<NT, MODE, U, VAR>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  select_compact_kernel<NT, MODE, U, VAR><<<(unsigned)(n_seg_req * p.layers * p.hkv), NT, smem, s>>>(
+      p, keys_cap);
+  return cudaGetLastError();
+}
+
+template <int NT, int U, int MODE>
+cudaError_t launch_var(const SelectCompactParams &p, int var, int n_seg_req, int keys_cap, size_t smem,
+                       cudaStream_t s) {
+  switch (var) {
+    case kOrderedSlotTie: return launch_one<NT, U, MODE, kOrderedSlotTie>(p, n_seg_req, keys_cap, smem, s);
+    case kOrderedPosTie: return launch_one<NT, U, MODE, kOrderedPosTie>(p, n_seg_req, keys_cap, smem, s);
+    default: return launch_one<NT, U, MODE, kHoleFill>(p, n_seg_req, keys_cap, smem, s);
+  }
 }
 
 template <int NT, int U>
-cudaError_t launch_nt(const SelectCompactParams &p, int mode, int n_seg_req, int max_n,
+cudaError_t launch_nt(const SelectCompactParams &p, int mode, int var, int n_seg_req, int max_n,
                       cudaStream_t s) {
   const int keys_cap = (max_n + 7) & ~7;
   const size_t smem = (size_t)keys_cap * (sizeof(uint32_t) + sizeof(uint16_t));
-  const dim3 grid((unsigned)(n_seg_req * p.layers * p.hkv));
-  cudaError_t e = cudaSuccess;
   switch (mode) {
-    case kModeRandom:
-      e = cudaFuncSetAttribute(select_compact_kernel<NT, kModeRandom, U>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess)
-        select_compact_kernel<NT, kModeRandom, U><<<grid, NT, smem, s>>>(p, keys_cap);
-      break;
-    case kModeRandomShared:
-      e = cudaFuncSetAttribute(select_compact_kernel<NT, kModeRandomShared, U>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess)
-        select_compact_kernel<NT, kModeRandomShared, U><<<grid, NT, smem, s>>>(p, keys_cap);
-      break;
-    default:
-      e = cudaFuncSetAttribute(select_compact_kernel<NT, kModeScores, U>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess)
-        select_compact_kernel<NT, kModeScores, U><<<grid, NT, smem, s>>>(p, keys_cap);
-      break;
+    case kModeRandom: return launch_var<NT, U, kModeRandom>(p, var, n_seg_req, keys_cap, smem, s);
+    case kModeRandomShared: return launch_var<NT, U, kModeRandomShared>(p, var, n_seg_req, keys_cap, smem, s);
+    default: return launch_var<NT, U, kModeScores>(p, var, n_seg_req, keys_cap, smem, s);
   }
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
 }
 
 }  // namespace
@@ -271,8 +389,9 @@ cudaError_t launch_select_compact(const SelectCompactParams &p, int mode, int n_
                                   int max_n, int max_m, cudaStream_t s) {
   (void)max_m;
   if (n_seg_req <= 0) return cudaSuccess;
-  if (max_n <= 4096) return launch_nt<256, KVC_SC_UNROLL_SMALL>(p, mode, n_seg_req, max_n, s);
-  return launch_nt<512, KVC_SC_UNROLL_LARGE>(p, mode, n_seg_req, max_n, s);
+  const int var = (p.flags & kScHoleFill) ? kHoleFill : (p.flags & kScTieByPos) ? kOrderedPosTie : kOrderedSlotTie;
+  if (max_n <= 4096) return launch_nt<256, KVC_SC_UNROLL_SMALL>(p, mode, var, n_seg_req, max_n, s);
+  return launch_nt<512, KVC_SC_UNROLL_LARGE>(p, mode, var, n_seg_req, max_n, s);
 }
 
 }  // namespace kvc

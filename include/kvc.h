@@ -227,6 +227,66 @@ kvc_status kvc_update_beacons(kvc_ctx *ctx, int32_t *assign_out, float *ms_out);
 kvc_status kvc_compress(kvc_ctx *ctx, kvc_selector selector, const int32_t *budgets,
                         uint64_t seed, void *debug_scores, kvc_round_stats *stats);
 
+/* Options of one eviction round (kvc_compress_ex).  The all-default value,
+ * {-1, 1, KVC_COMPACT_ORDERED, 0}, is the round of kvc_compress.
+ *   sink_tokens: < 0 protects the whole prompt.  S >= 0 protects only the
+ *     first min(P, S) positions, the attention sinks, as the SnapKV-style
+ *     baselines of the Random Attention article do ("发现一", on protection
+ *     regimes); the rest of the prompt competes with the generated
+ *     positions, and the request's protected length becomes min(P, S) for
+ *     later rounds once a round evicts from it.
+ *   block: random selectors only (must be 1 for the beacon selector),
+ *     1 <= block <= 32768: the positions of one block, pos / block, share one
+ *     Philox draw (counter word 0 = pos / block), so whole blocks are kept in
+ *     order of their draw and at most one block is split, at its lowest
+ *     positions ("发现二": contiguous blocks of 1 to 256 tokens).
+ *   compaction: KVC_COMPACT_ORDERED packs the survivors in slot order;
+ *     KVC_COMPACT_HOLE_FILL leaves every survivor below the new length in
+ *     place and moves the i-th survivor at or past it into the i-th evicted
+ *     slot below it (ascending), copying only as many rows as there are
+ *     holes.  Slots then no longer follow position order; later rounds still
+ *     rank ties by original position and keep slot order among survivors.
+ *   reserved: 0. */
+typedef enum kvc_compaction { KVC_COMPACT_ORDERED = 0, KVC_COMPACT_HOLE_FILL = 1 } kvc_compaction;
+
+typedef struct kvc_round_options {
+  int32_t sink_tokens;
+  int32_t block;
+  int32_t compaction;
+  int32_t reserved;
+} kvc_round_options;
+
+/* kvc_compress with round options; opts NULL means the defaults.  Invalid
+ * options return KVC_ERR_INVALID_ARG with nothing enqueued. */
+kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *budgets,
+                           uint64_t seed, const kvc_round_options *opts, void *debug_scores,
+                           kvc_round_stats *stats);
+
+/* One decode step of attention over the cache as it stands (after any
+ * eviction round), for layers [layer_begin, layer_begin + layer_count): the
+ * attention kernels every selector shares in the Random Attention article's
+ * serving setup ("发现四"; eviction only changes which rows they read).  For
+ * request r, layer l and query head hq, with h = hq / G the KV head it reads
+ * (G = num_q_heads / num_kv_heads, as in the beacon update):
+ *     s_j = scale * q . k_j over the request's cached rows j < length(r),
+ *     out = sum_j exp(s_j - lse) v_j,   lse = log sum_j exp(s_j).
+ * Slot order does not matter (rows after hole filling included).  A request
+ * with no rows gets out = 0 and lse = -inf.
+ *   q:   device [layer_count][num_requests][num_q_heads][head_dim] in the
+ *        cache dtype, element-aligned; read only.
+ *   scale: > 0, or 0 for 1/sqrt(head_dim).
+ *   out: device float [layer_count][num_requests][num_q_heads][head_dim].
+ *   lse: device float [layer_count][num_requests][num_q_heads] or NULL
+ *        (natural log).
+ *   ms_out: host float or NULL; if given, the call synchronises and writes
+ *     the device time of its kernels, and reports latched device errors.
+ * Enqueued on the context's stream; uses the context's workspace for split
+ * partials, so calls on one context must not overlap.  Errors (nothing
+ * enqueued): KVC_ERR_INVALID_ARG; KVC_ERR_UNSUPPORTED unless the cache is
+ * bf16 or f32 with head_dim 64 or 128 and G in {1, 2, 4, 8}. */
+kvc_status kvc_decode_attention(kvc_ctx *ctx, int32_t layer_begin, int32_t layer_count, const void *q,
+                                float scale, float *out, float *lse, float *ms_out);
+
 /* Fills *out with device pointers to the live state (no copy, no sync). */
 kvc_status kvc_gather_view(const kvc_ctx *ctx, kvc_view *out);
 

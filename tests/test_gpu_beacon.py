@@ -45,7 +45,7 @@ def _fill_recording(ctx, w, gen):
     return qwin
 
 
-def run_beacon(w, sample=None, score_impl=None):
+def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered"):
     ctx = make_context(w)
     if score_impl is not None:
         ctx.set_option(0, score_impl)
@@ -104,7 +104,8 @@ def run_beacon(w, sample=None, score_impl=None):
             pre[l] = (full_pos, full_k, full_v)
     scores = torch.zeros((R, Ly, H, ctx.spec.max_seq_len), dtype=torch.float32, device="cuda")
     budgets = w.budget.astype(np.int32)
-    stats = ctx.compress("beacon", budgets, w.philox_seed, debug_scores=scores, stats=True)
+    stats = ctx.compress("beacon", budgets, w.philox_seed, debug_scores=scores, stats=True,
+                         sink_tokens=sinks, compaction=compaction)
     ctx.sync()
     new_len, _ = ctx.lengths()
     g_scores = scores.cpu().numpy()
@@ -112,6 +113,8 @@ def run_beacon(w, sample=None, score_impl=None):
     differ = in_abs = in_rel = 0
     for (r, l, h) in segs:
         L, P, K = int(lengths[r]), int(prompts[r]), int(budgets[r])
+        if sinks is not None:
+            P = min(P, sinks)
         keys = pre[l][1][r, h, :L].float().cpu().numpy().astype(np.float64)
         o_sc, _ = oracle.beacon_score(keys, g_scoring[r, l, h], P)
         if L <= K:
@@ -125,7 +128,10 @@ def run_beacon(w, sample=None, score_impl=None):
         gpu_kept = np.searchsorted(pre[l][0][r, h, :L], post_pos[0, h])
         assert np.array_equal(pre[l][0][r, h, gpu_kept], post_pos[0, h])
         assert np.array_equal(gpu_kept[:P], np.arange(P))
-        dd, ia, ir = band_check(gpu_kept[P:], o_sc, P, M, N)
+        if compaction == "hole_fill":
+            # same kept set as order-preserving compaction, laid out by hole filling
+            assert np.array_equal(gpu_kept, oracle.hole_fill(P + M, np.sort(gpu_kept)))
+        dd, ia, ir = band_check(np.sort(gpu_kept)[P:], o_sc, P, M, N)
         differ += dd
         in_abs += ia
         in_rel += ir
@@ -157,6 +163,13 @@ def test_long_trace_sampled():
     w = wl.scaled(wl.long_trace(), num_requests=2, num_layers=4)
     out = run_beacon(w, sample=3)
     print(out)
+
+
+@pytest.mark.parametrize("sinks,compaction", [(4, "ordered"), (None, "hole_fill"), (0, "hole_fill")])
+def test_beacon_round_options(sinks, compaction):
+    """Sink-only protection and hole-filling compaction under the beacon selector."""
+    out = run_beacon(wl.beacon_serving(R=3, layers=2), sinks=sinks, compaction=compaction)
+    print(sinks, compaction, out)
 
 
 @pytest.mark.parametrize("impl", [1, 2], ids=["simt", "tcgen05"])
