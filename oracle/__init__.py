@@ -45,6 +45,8 @@ PINS = {
     "random_score_block": "numpy.random.Philox on counter (pos // block, h, l, r)",
     "hole_fill": "invariants: kept slots below R stay, holes filled in ascending order, same kept set",
     "random_round_ex": "at most one split block; sink protection = prompt protection with P = S",
+    "beacon_trigger_score": "scipy.special.softmax weighted by trigger shares; one-hot trigger -> that "
+                            "beacon's softmax; mass conservation sum_j = 1 (P = 0); count scaling invariance",
     "decode_attention": "scipy.special.softmax/logsumexp; L=1 -> v; q=0 -> mean of v, log L; "
                         "large-scale limit -> v of the argmax key; joint permutation invariance",
     "decode_attention_gqa": "query head hq reads KV head hq // G (marker values per KV head)",
@@ -96,6 +98,8 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.orc_random_round_segment_ex.restype = i64
     L.orc_random_round_batch_ex.argtypes = [u64, u64, i32, i64, i32, i64, P, P, i64, P, P, P]
     L.orc_random_round_batch_ex.restype = i64
+    L.orc_beacon_trigger_score.argtypes = [i64, i64, i64, i64, P, P, P, P]
+    L.orc_beacon_trigger_score.restype = i32
     L.orc_decode_attention.argtypes = [i64, i64, P, P, P, ctypes.c_double, P, P]
     L.orc_decode_attention.restype = None
     L.orc_decode_attention_gqa.argtypes = [i64, i64, i64, i64, P, P, P, ctypes.c_double, P, P]
@@ -379,3 +383,16 @@ def decode_attention_gqa(q, k, v, scale=None):
     lse = np.zeros(Hq, np.float64)
     lib().orc_decode_attention_gqa(Hq, Hkv, L, d, _ptr(q), _ptr(k), _ptr(v), scale, _ptr(out), _ptr(lse))
     return out, lse
+
+
+def beacon_trigger_score(keys, beacons_scoring, trig, P: int):
+    """Cluster-trigger importance [L-P] of one segment (keys [L,d], beacons [B,d], trig [B])."""
+    k = np.ascontiguousarray(keys, dtype=np.float64)
+    c = np.ascontiguousarray(beacons_scoring, dtype=np.float64)
+    t = np.ascontiguousarray(trig, dtype=np.float64)
+    L, d = k.shape
+    B = c.shape[0]
+    score = np.zeros(max(L - P, 1), np.float64)
+    if lib().orc_beacon_trigger_score(L, P, B, d, _ptr(k), _ptr(c), _ptr(t), _ptr(score)) != 0:
+        raise ValueError("beacon_trigger_score failed")
+    return score[:L - P]

@@ -518,6 +518,60 @@ int32_t orc_beacon_score(int64_t L, int64_t P, int64_t B, int64_t d, const doubl
 }
 
 /* ------------------------------------------------------------------ */
+/* BeaconKV cluster-level trigger (the build's reading of [BX] §3.2:   */
+/* "query -> cluster -> KV" and mark_important(cluster_id, KV)).       */
+/* ------------------------------------------------------------------ */
+
+/* Each query of the latest update window lands in one cluster (its nearest
+ * beacon); the trigger raises the importance of the keys that cluster's
+ * beacon attends to.  With m_b the number of window queries assigned to
+ * beacon b and z_bj, lse_b as in orc_beacon_score:
+ *     importance_j = sum_b (m_b / sum_b' m_b') * exp(z_bj - lse_b),  j in [P, L)
+ * i.e. the attention mass key j receives when every window query is replaced
+ * by its cluster's beacon.  All m_b = 0 gives importance 0 everywhere.
+ * keys [L][d], beacons [B][d], trig [B] (counts, >= 0); score_out[0..L-P). */
+int32_t orc_beacon_trigger_score(int64_t L, int64_t P, int64_t B, int64_t d, const double *keys,
+                                 const double *beacons, const double *trig, double *score_out) {
+  if (L <= 0 || P < 0 || P > L || B <= 0 || d <= 0) return -1;
+  double total = 0.0;
+  for (int64_t b = 0; b < B; ++b) {
+    if (trig[b] < 0) return -1;
+    total += trig[b];
+  }
+  double *z = (double *)malloc((size_t)(B * L) * sizeof(double));
+  double *lse = (double *)malloc((size_t)B * sizeof(double));
+  if (!z || !lse) {
+    free(z);
+    free(lse);
+    return -1;
+  }
+  const double rsqrt_d = 1.0 / sqrt((double)d);
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t j = 0; j < L; ++j) {
+      double dot = 0.0;
+      for (int64_t k = 0; k < d; ++k) dot += beacons[b * d + k] * keys[j * d + k];
+      z[b * L + j] = dot * rsqrt_d;
+    }
+  for (int64_t b = 0; b < B; ++b) {
+    double mx = -INFINITY;
+    for (int64_t j = 0; j < L; ++j)
+      if (z[b * L + j] > mx) mx = z[b * L + j];
+    double sum = 0.0;
+    for (int64_t j = 0; j < L; ++j) sum += exp(z[b * L + j] - mx);
+    lse[b] = mx + log(sum);
+  }
+  for (int64_t j = P; j < L; ++j) {
+    double acc = 0.0;
+    if (total > 0)
+      for (int64_t b = 0; b < B; ++b) acc += (trig[b] / total) * exp(z[b * L + j] - lse[b]);
+    score_out[j - P] = acc;
+  }
+  free(z);
+  free(lse);
+  return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* Decode attention over a request's cached rows [RA, "发现四": every     */
 /* selector shares the same paged attention kernels; what they attend  */
 /* to is the compacted cache].                                         */

@@ -313,6 +313,38 @@ def check_random_round_ex():
             assert len(out) == K and np.array_equal(out[:P], pos_in[:P])
 
 
+def check_beacon_trigger_score():
+    from scipy.special import softmax
+    rng = np.random.default_rng(31)
+    for (L, P, B, d) in [(40, 4, 3, 8), (64, 0, 5, 16), (33, 10, 1, 32)]:
+        keys = rng.standard_normal((L, d))
+        bea = rng.standard_normal((B, d))
+        trig = rng.integers(0, 20, B).astype(np.float64)
+        trig[0] += 1
+        sc = oracle.beacon_trigger_score(keys, bea, trig, P)
+        A = softmax(bea @ keys.T / np.sqrt(d), axis=1)  # [B, L]
+        want = (trig / trig.sum()) @ A
+        assert np.allclose(sc, want[P:], rtol=1e-12, atol=1e-15)
+        # scaling the counts changes nothing
+        assert np.allclose(oracle.beacon_trigger_score(keys, bea, 7 * trig, P), sc, rtol=1e-13, atol=0)
+        # one-hot trigger: that beacon's attention row
+        b = int(rng.integers(B))
+        oh = np.zeros(B)
+        oh[b] = 3
+        assert np.allclose(oracle.beacon_trigger_score(keys, bea, oh, P), A[b, P:], rtol=1e-12, atol=1e-15)
+    # mass conservation over all keys (P = 0)
+    keys = rng.standard_normal((50, 8))
+    sc = oracle.beacon_trigger_score(keys, rng.standard_normal((4, 8)), np.array([1.0, 0, 5, 2]), 0)
+    assert abs(sc.sum() - 1.0) <= 1e-12
+    # identical keys: 1/L whatever the beacons and triggers
+    keys = np.tile(rng.standard_normal(8), (25, 1))
+    sc = oracle.beacon_trigger_score(keys, rng.standard_normal((3, 8)), np.array([2.0, 1, 0]), 5)
+    assert np.allclose(sc, 1 / 25, rtol=1e-12)
+    # no trigger at all: zeros
+    sc = oracle.beacon_trigger_score(keys, rng.standard_normal((3, 8)), np.zeros(3), 5)
+    assert np.array_equal(sc, np.zeros(20))
+
+
 def check_decode_attention():
     from scipy.special import logsumexp, softmax
     rng = np.random.default_rng(23)
@@ -366,4 +398,4 @@ def check_decode_attention_gqa():
 ALL = [check_philox, check_random_score, check_retention, check_select, check_compact,
        check_random_round_invariants, check_survival, check_head_independence, check_bf16,
        check_beacon_update, check_beacon_score, check_block_score, check_hole_fill, check_random_round_ex,
-       check_decode_attention, check_decode_attention_gqa]
+       check_decode_attention, check_decode_attention_gqa, check_beacon_trigger_score]

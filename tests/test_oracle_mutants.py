@@ -48,6 +48,14 @@ MUTANTS = [
      [pins.check_block_score]),
     ("hole_fill_reverse", "for (int64_t i = 0; i < R; ++i) {\n    if (kept_slots[i] < R) continue;",
      "for (int64_t i = R - 1; i >= 0; --i) {\n    if (kept_slots[i] < R) continue;", [pins.check_hole_fill]),
+    ("trigger_unnormalised", "acc += (trig[b] / total) * exp(z[b * L + j] - lse[b]);",
+     "acc += trig[b] * exp(z[b * L + j] - lse[b]);", [pins.check_beacon_trigger_score]),
+    ("trigger_max_not_sum", "acc += (trig[b] / total) * exp(z[b * L + j] - lse[b]);",
+     "acc = fmax(acc, (trig[b] / total) * exp(z[b * L + j] - lse[b]));", [pins.check_beacon_trigger_score]),
+    ("trigger_lse_skips_prompt", "for (int64_t j = 0; j < L; ++j) sum += exp(z[b * L + j] - mx);",
+     "for (int64_t j = P; j < L; ++j) sum += exp(z[b * L + j] - mx);", [pins.check_beacon_trigger_score]),
+    ("trigger_scale_by_d", "const double rsqrt_d = 1.0 / sqrt((double)d);", "const double rsqrt_d = 1.0 / (double)d;",
+     [pins.check_beacon_trigger_score]),
     ("attention_no_scale", "s[j] = scale * dot;", "s[j] = dot;", [pins.check_decode_attention]),
     ("attention_lse_drops_max", "double lse = mx + log(sum);", "double lse = log(sum);",
      [pins.check_decode_attention]),
