@@ -102,7 +102,7 @@ def make_workload(args):
     if kw:
         w = wl.scaled(w, **kw)
     sel = args.selector or w.selectors[0]
-    if sel != "beacon" and w.num_beacons:
+    if sel not in ("beacon", "beacon_trigger") and w.num_beacons:
         w = wl.scaled(w, num_beacons=0, query_window=0, num_q_heads=w.num_kv_heads)
     return w, sel
 
@@ -265,14 +265,14 @@ def run_ours(args, rank, world, dist):
                        num_q_heads=w.num_q_heads or w.num_kv_heads, num_beacons=w.num_beacons,
                        query_window=w.query_window)
     ctx = Context(spec, dtype=wl.torch_dtype(w.dtype), device=dev)
-    if sel == "beacon" and args.score_impl:
+    if sel in ("beacon", "beacon_trigger") and args.score_impl:
         ctx.set_option(0, args.score_impl)
     gen = wl.Generator(w, dev)
     wl.fill(ctx, w, gen)
     budgets = w.budget.astype(np.int32)
     R = w.num_requests
     ids = np.arange(R, dtype=np.int32)
-    beacon = sel == "beacon"
+    beacon = sel in ("beacon", "beacon_trigger")
     T = w.trigger
     refill = Refill(ctx, w, gen)
 
@@ -588,8 +588,8 @@ def oracle_sample_rate(w, sel, budget_s: float, rank_seed: int = 0):
         if key not in cache:
             rows_k = rng.integers(0, 255, (L, d * es), dtype=np.uint8)
             rows_v = rng.integers(0, 255, (L, d * es), dtype=np.uint8)
-            keys = rng.standard_normal((L, d)) if sel == "beacon" else None
-            pts = rng.standard_normal((w.query_window * w.G, d)) if sel == "beacon" else None
+            keys = rng.standard_normal((L, d)) if sel.startswith("beacon") else None
+            pts = rng.standard_normal((w.query_window * w.G, d)) if sel.startswith("beacon") else None
             cache[key] = (rows_k, rows_v, keys, pts)
         rows_k, rows_v, keys, pts = cache[key]
         pos = np.arange(L, dtype=np.int32)
@@ -597,6 +597,10 @@ def oracle_sample_rate(w, sel, budget_s: float, rank_seed: int = 0):
         if sel == "beacon":
             c, cnt, _ = oracle.beacon_update(pts, np.zeros((w.num_beacons, d)), np.zeros(w.num_beacons), init=True)
             kept, _ = oracle.beacon_round_segment(keys, P, K, oracle.round_bf16(c) if w.dtype == "bf16" else c)
+        elif sel == "beacon_trigger":
+            c, cnt, _ = oracle.beacon_update(pts, np.zeros((w.num_beacons, d)), np.zeros(w.num_beacons), init=True)
+            sc = oracle.beacon_trigger_score(keys, oracle.round_bf16(c) if w.dtype == "bf16" else c, cnt, P)
+            kept = oracle.beacon_select_with_pos(sc.astype(np.float32), pos, P, K)
         else:
             kept, _ = oracle.random_round_segment(w.philox_seed, 0, r, l, h, sel == "random_shared", P, K, pos)
         oracle.compact_rows(rows_k, P, kept[P:])

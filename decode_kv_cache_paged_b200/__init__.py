@@ -45,6 +45,7 @@ KVC_F32 = 1
 KVC_SEL_RANDOM = 0
 KVC_SEL_RANDOM_SHARED = 1
 KVC_SEL_BEACON = 2
+KVC_SEL_BEACON_TRIGGER = 3
 
 KVC_OPT_BEACON_SCORE_IMPL = 0
 KVC_OPT_BEACON_UPDATE_IMPL = 1
@@ -54,7 +55,7 @@ KVC_COMPACT_HOLE_FILL = 1
 COMPACTIONS = {"ordered": KVC_COMPACT_ORDERED, "hole_fill": KVC_COMPACT_HOLE_FILL}
 
 SELECTORS = {"random": KVC_SEL_RANDOM, "random_shared": KVC_SEL_RANDOM_SHARED,
-             "beacon": KVC_SEL_BEACON}
+             "beacon": KVC_SEL_BEACON, "beacon_trigger": KVC_SEL_BEACON_TRIGGER}
 
 
 class kvc_config(ctypes.Structure):
@@ -91,6 +92,7 @@ class kvc_view(ctypes.Structure):
                 ("prompt_lengths", ctypes.c_void_p), ("pos_map", ctypes.c_void_p),
                 ("query_ring", ctypes.c_void_p), ("beacons", ctypes.c_void_p),
                 ("beacons_scoring", ctypes.c_void_p), ("beacon_counts", ctypes.c_void_p),
+                ("beacon_triggers", ctypes.c_void_p),
                 ("max_pages_per_request", ctypes.c_int32), ("row_bytes", ctypes.c_int32),
                 ("round", ctypes.c_int64)]
 
@@ -313,6 +315,8 @@ class Context:
             out["beacons_scoring"] = self._ws_tensor(v.beacons_scoring, R * Ly * H * B * d * es, self.dtype,
                                                      (R, Ly, H, B, d))
             out["beacon_counts"] = self._ws_tensor(v.beacon_counts, R * Ly * H * B * 4, torch.int32, (R, Ly, H, B))
+            out["beacon_triggers"] = self._ws_tensor(v.beacon_triggers, R * Ly * H * B * 4, torch.float32,
+                                                     (R, Ly, H, B))
         return out
 
     def gather_dense(self, layer: int, req_begin: int = 0, req_count: int | None = None, cap: int | None = None):

@@ -61,6 +61,7 @@ struct TcParams {
   const SegDesc *segs;
   float *scores;
   float *lse_out;
+  const float *trig;  // cluster-trigger shares [seg][B], or null for the max rule
   int32_t *status;
   int64_t num_pages;
   int32_t bt_stride, layers, hkv, B, max_seq, n_segs;
@@ -106,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     beacon_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap cmap,
                            TcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *smem = smem_align<1024>(smem_raw);
   constexpr uint32_t kCBytes = CROWS * 256;          // beacon tile: CROWS rows x 128 bf16
   constexpr uint32_t kTileBytes = kTileKeys * 256;   // 32 KB
   uint8_t *cbuf = smem;                              // [NCB][2 K-halves][CROWS][128 B]
@@ -120,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *lse2 = reinterpret_cast<float *>(tmem_slot + 4);  // [2][256]
   float *part = lse2 + 512;                                 // [4][2][256] partial (m, sum)
+  float *wts2 = part + 4 * 2 * 256;                         // [2][256] trigger shares
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -288,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = blockIdx.x; s < p.n_segs && ok; s += gridDim.x, ++si) {
       const SegGeom g = seg_geom<kStages>(p, s);
       float *lse_buf = lse2 + (si & 1) * 256;
+      float *w_buf = wts2 + (si & 1) * 256;
       // pass 1: per-beacon online log2-sum-exp2 over this group's tiles
       float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
       for (int t = 0; t < g.n1; ++t, ++acc_it) {
@@ -359,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float l2 = mm + log2f(ss);
             lse_buf[b] = l2;
+            if (p.trig) w_buf[b] = p.trig[g.seg_flat * B + b];
             if (p.lse_out) p.lse_out[g.seg_flat * B + b] = l2 * 0.69314718055994531f;
             if (l2 != l2) atomicCAS(p.status, kDevOk, kDevNaN);
           }
@@ -378,19 +382,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tmem_fence_after();
         float bm[8];
+        const bool trig = p.trig != nullptr;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) bm[i] = -INFINITY;
+        for (int i = 0; i < 8; ++i) bm[i] = trig ? 0.f : -INFINITY;
         for (int c0 = 0; c0 < B; c0 += 64) {
           float v[64];
           tmem_ld64(tmem_base + lane_addr + buf * 256 + c0, v);
           const float4 *l4 = reinterpret_cast<const float4 *>(lse_buf + c0);
+          if (trig) {
+            // cluster trigger: sum over beacons of share_b * 2^(u_bj - lse2_b)
+            const float4 *w4 = reinterpret_cast<const float4 *>(w_buf + c0);
 #pragma unroll
-          for (int i4 = 0; i4 < 16; ++i4) {
-            const float4 L4 = l4[i4];
-            bm[(4 * i4) & 7] = fmaxf(bm[(4 * i4) & 7], fmaf(v[4 * i4], alpha, -L4.x));
-            bm[(4 * i4 + 1) & 7] = fmaxf(bm[(4 * i4 + 1) & 7], fmaf(v[4 * i4 + 1], alpha, -L4.y));
-            bm[(4 * i4 + 2) & 7] = fmaxf(bm[(4 * i4 + 2) & 7], fmaf(v[4 * i4 + 2], alpha, -L4.z));
-            bm[(4 * i4 + 3) & 7] = fmaxf(bm[(4 * i4 + 3) & 7], fmaf(v[4 * i4 + 3], alpha, -L4.w));
+            for (int i4 = 0; i4 < 16; ++i4) {
+              const float4 L4 = l4[i4], W4 = w4[i4];
+              bm[(4 * i4) & 7] = fmaf(W4.x, exp2f(fmaf(v[4 * i4], alpha, -L4.x)), bm[(4 * i4) & 7]);
+              bm[(4 * i4 + 1) & 7] = fmaf(W4.y, exp2f(fmaf(v[4 * i4 + 1], alpha, -L4.y)), bm[(4 * i4 + 1) & 7]);
+              bm[(4 * i4 + 2) & 7] = fmaf(W4.z, exp2f(fmaf(v[4 * i4 + 2], alpha, -L4.z)), bm[(4 * i4 + 2) & 7]);
+              bm[(4 * i4 + 3) & 7] = fmaf(W4.w, exp2f(fmaf(v[4 * i4 + 3], alpha, -L4.w)), bm[(4 * i4 + 3) & 7]);
+            }
+          } else {
+#pragma unroll
+            for (int i4 = 0; i4 < 16; ++i4) {
+              const float4 L4 = l4[i4];
+              bm[(4 * i4) & 7] = fmaxf(bm[(4 * i4) & 7], fmaf(v[4 * i4], alpha, -L4.x));
+              bm[(4 * i4 + 1) & 7] = fmaxf(bm[(4 * i4 + 1) & 7], fmaf(v[4 * i4 + 1], alpha, -L4.y));
+              bm[(4 * i4 + 2) & 7] = fmaxf(bm[(4 * i4 + 2) & 7], fmaf(v[4 * i4 + 2], alpha, -L4.z));
+              bm[(4 * i4 + 3) & 7] = fmaxf(bm[(4 * i4 + 3) & 7], fmaf(v[4 * i4 + 3], alpha, -L4.w));
+            }
           }
         }
         tmem_fence_before();
@@ -398,9 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
         const int j = g.tile_of(g.n1 + t) * kTileKeys + row;
         if (j >= g.P && j < g.L) {
-          const float best = fmaxf(fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3])),
-                                   fmaxf(fmaxf(bm[4], bm[5]), fmaxf(bm[6], bm[7])));
-          const float sc = exp2f(best);
+          const float sc =
+              trig ? ((bm[0] + bm[1]) + (bm[2] + bm[3])) + ((bm[4] + bm[5]) + (bm[6] + bm[7]))
+                   : exp2f(fmaxf(fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3])),
+                                 fmaxf(fmaxf(bm[4], bm[5]), fmaxf(bm[6], bm[7]))));
           if (sc != sc) atomicCAS(p.status, kDevOk, kDevNaN);
           p.scores[g.seg_flat * p.max_seq + (j - g.P)] = sc;
         }
@@ -443,7 +462,7 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows
 template <int CROWS, int NCB, int kStages>
 cudaError_t launch(const CUtensorMap &km, const CUtensorMap &cm, const TcParams &tp, cudaStream_t s) {
   const size_t smem = 1024 + (size_t)NCB * CROWS * 256 + (size_t)kStages * kTileKeys * 256 + 256 +
-                      2 * 256 * 4 + 4 * 2 * 256 * 4;
+                      2 * 256 * 4 + 4 * 2 * 256 * 4 + 2 * 256 * 4;
   cudaError_t e = cudaFuncSetAttribute(beacon_score_tc_kernel<CROWS, NCB, kStages>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -477,6 +496,7 @@ cudaError_t launch_beacon_score_tc(const BeaconScoreParams &p, int n_req, int ma
   tp.segs = p.segs;
   tp.scores = p.scores;
   tp.lse_out = p.lse_out;
+  tp.trig = p.trig;
   tp.status = p.status;
   tp.num_pages = p.num_pages;
   tp.bt_stride = p.bt_stride;

@@ -221,7 +221,10 @@ __global__ void __launch_bounds__(kUpdNT) beacon_update_kernel(BeaconUpdateParam
       gbeac[e] = v;
       store_scoring<DT>(p.beacons_s, seg * p.B * D + e, v);
     }
-    if (lane == 0) gcnt[b] = n + m;
+    if (lane == 0) {
+      gcnt[b] = n + m;
+      p.trig[seg * p.B + b] = (float)m / (float)n_pts;
+    }
   }
 }
 
@@ -239,6 +242,7 @@ __global__ void __launch_bounds__(kScNT) beacon_score_simt_kernel(BeaconScorePar
   float *zs = ks + kTK * (D + 1);                // [B][kTK+1]
   float *lse = zs + p.B * (kTK + 1);             // [B]
   float *red = lse + p.B;                        // [kNG][kTK]
+  float *wts = red + kNG * kTK;                   // [B] trigger shares (cluster-trigger mode)
   const int tid = threadIdx.x;
   const int h = blockIdx.x % p.hkv;
   const int l = (blockIdx.x / p.hkv) % p.layers;
@@ -250,6 +254,8 @@ __global__ void __launch_bounds__(kScNT) beacon_score_simt_kernel(BeaconScorePar
 
   for (int e = tid; e < p.B * D; e += kScNT)
     cs[e] = load_elem<DT>(p.beacons_s, seg * p.B * D + e);
+  if (p.trig)
+    for (int e = tid; e < p.B; e += kScNT) wts[e] = p.trig[seg * p.B + e];
 
   const int jj = tid % kTK, bg = tid / kTK;
   auto load_tile = [&](int j0) {
@@ -303,7 +309,8 @@ __global__ void __launch_bounds__(kScNT) beacon_score_simt_kernel(BeaconScorePar
     if (v != v) set_status(p.status, kDevNaN);
   }
 
-  // pass 2: per candidate key, max over beacons of z - lse
+  // pass 2: per candidate key, max over beacons of z - lse (or the
+  // trigger-weighted sum of the beacons' attention on it)
 #pragma unroll 1
   for (int j0 = P; j0 < L; j0 += kTK) {
     __syncthreads();
@@ -311,14 +318,27 @@ __global__ void __launch_bounds__(kScNT) beacon_score_simt_kernel(BeaconScorePar
     __syncthreads();
     dots();
     __syncthreads();
-    float mx = __int_as_float(0xff800000);
-    for (int b = bg; b < p.B; b += kNG) mx = fmaxf(mx, zs[b * (kTK + 1) + jj] - lse[b]);
-    red[bg * kTK + jj] = mx;
+    if (p.trig) {
+      // cluster trigger: sum over beacons of share_b * exp(z - lse_b)
+      float acc = 0.f;
+      for (int b = bg; b < p.B; b += kNG) acc = fmaf(wts[b], expf(zs[b * (kTK + 1) + jj] - lse[b]), acc);
+      red[bg * kTK + jj] = acc;
+    } else {
+      float mx = __int_as_float(0xff800000);
+      for (int b = bg; b < p.B; b += kNG) mx = fmaxf(mx, zs[b * (kTK + 1) + jj] - lse[b]);
+      red[bg * kTK + jj] = mx;
+    }
     __syncthreads();
     if (tid < kTK && j0 + tid < L) {
       float m = red[tid];
-      for (int g = 1; g < kNG; ++g) m = fmaxf(m, red[g * kTK + tid]);
-      const float sc = expf(m);
+      float sc;
+      if (p.trig) {
+        for (int g = 1; g < kNG; ++g) m += red[g * kTK + tid];
+        sc = m;
+      } else {
+        for (int g = 1; g < kNG; ++g) m = fmaxf(m, red[g * kTK + tid]);
+        sc = expf(m);
+      }
       if (sc != sc) set_status(p.status, kDevNaN);
       p.scores[seg * p.max_seq + (j0 + tid - P)] = sc;
     }
@@ -352,7 +372,7 @@ cudaError_t launch_beacon_score_simt(const BeaconScoreParams &p, int n_req, cuda
   if (n_req <= 0) return cudaSuccess;
   const unsigned grid = (unsigned)(n_req * p.layers * p.hkv);
   const size_t smem = sizeof(float) * ((size_t)p.B * p.d + (size_t)kTK * (p.d + 1) +
-                                       (size_t)p.B * (kTK + 1) + p.B + kNG * kTK);
+                                       (size_t)p.B * (kTK + 1) + p.B + kNG * kTK + p.B);
   cudaError_t e = cudaErrorInvalidValue;
 #define KVC_SC(DV, DTV)                                                                       \
   if (p.d == DV && p.dtype == DTV) {                                                          \

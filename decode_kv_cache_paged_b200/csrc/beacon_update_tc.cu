@@ -36,7 +36,7 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int k) {
 
 __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParams p, uint32_t tmem_cols) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *smem = smem_align<1024>(smem_raw);
   constexpr int D = 128;
   const int B = p.B, NP = p.W * p.G;
   uint8_t *xs = smem;                    // [2 K-blocks][128 rows][128 B]
@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
   int32_t *order = assign + NP;                                   // [NP]
   int32_t *offs = order + NP;                                     // [B + 1]
   int32_t *cursor = offs + B + 1;                                 // [B]
-  uint64_t *mbar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(cursor + B) + 15) & ~uintptr_t(15));
+  uint64_t *mbar = smem_align<16>(reinterpret_cast<uint64_t *>(cursor + B));
   uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -245,7 +245,10 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
         gbeac[b * D + k] = v;
         reinterpret_cast<__nv_bfloat16 *>(p.beacons_s)[seg * B * D + b * D + k] = __float2bfloat16_rn(v);
       }
-      if (lane == 0) gcnt[b] = n + m;
+      if (lane == 0) {
+        gcnt[b] = n + m;
+        p.trig[seg * B + b] = (float)m / (float)n_pts;
+      }
     }
   }
   tmem_fence_before();
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
 // twice from global memory.
 __global__ void __launch_bounds__(kUT) beacon_update_tc_scatter_kernel(BeaconUpdateParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *smem = smem_align<1024>(smem_raw);
   constexpr int D = 128;
   constexpr uint32_t kCols = 256;        // [0, 128) assignment product, [128, 256) sums
   const int B = p.B, NP = p.W * p.G;
@@ -277,7 +280,7 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_scatter_kernel(BeaconUpd
   float *cn = reinterpret_cast<float *>(asum + 32768);  // [B]
   float *cpart = cn + B;                                 // [4][B]
   int32_t *cnt = reinterpret_cast<int32_t *>(cpart + 4 * B);  // [B]
-  uint64_t *mbar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(cnt + B) + 15) & ~uintptr_t(15));
+  uint64_t *mbar = smem_align<16>(reinterpret_cast<uint64_t *>(cnt + B));
   uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -467,6 +470,7 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_scatter_kernel(BeaconUpd
         s2[2 * k4 + 1] = __floats2bfloat162_rn(v[2], v[3]);
       }
       gcnt[b] = n + m;
+      p.trig[seg * B + b] = (float)m / (float)n_pts;
     }
   }
   tmem_fence_before();

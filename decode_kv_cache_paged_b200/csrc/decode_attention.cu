@@ -13,19 +13,21 @@
 // G query heads of its KV head only, 2G flop per element), so it runs on the
 // CUDA cores and spends its effort on keeping HBM busy.
 //   * Work unit = (layer, request, KV head, split of the pages); one CTA of
-//     128 threads each.  Splits give short batches enough CTAs; a second
-//     kernel merges the per-split (max, sum, output) partials.
-//   * Tiles of 4 pages (64 rows): the K and V rows of a page are 16
-//     consecutive pool rows, fetched by one elected thread as 2-D TMA tiles
-//     (128-byte boxes, 128-byte swizzle) into a ring of stages with
-//     transaction-count mbarriers, so loads of later tiles overlap compute.
-//   * Scores: two threads per row, each half the dimensions; with the
-//     swizzle, the 8 lanes of a quarter-warp read 8 different rows' chunks
-//     from 8 different bank groups while reading the same query chunk
-//     (broadcast).  Online softmax in base 2 with the scale folded into q.
-//   * P.V: each thread owns 8 bytes of a row (4 bf16 dimensions) for all G
-//     heads and walks a quarter of the tile's rows; the row groups are added
-//     at the end.
+//     4 warps each.  Splits give short batches enough CTAs; a second kernel
+//     merges the per-split (max, sum, output) partials.
+//   * Each warp walks every 4th page of the unit on its own: the K and V
+//     rows of a page are 16 consecutive pool rows, fetched as 2-D TMA tiles
+//     (128-byte boxes, 128-byte swizzle, one box per lane) into the warp's
+//     2-slot ring with transaction-count mbarriers.  Warps keep their own
+//     running max and sums, so no block-wide barrier is taken until the
+//     four warps' states are merged at the end.
+//   * Scores: two lanes per row, each half the dimensions; with the swizzle
+//     the 8 lanes of a quarter-warp read 8 rows' chunks from 8 different
+//     bank groups while reading the same query chunk (broadcast).  Online
+//     softmax in base 2 with the scale folded into q.
+//   * P.V: each lane owns 8-byte segments of a row for all G heads.
+//   * Products and sums use the packed two-wide fp32 FMA of sm_100 (the
+//     same rounding as two scalar FMAs, half the instructions).
 // Every mbarrier wait is bounded: on timeout the kernel records
 // kDevTimeout in the status word, lets its own copies land (bounded) and
 // leaves, all threads of the CTA together.
@@ -39,47 +41,48 @@
 namespace kvc {
 namespace {
 
+#ifndef KVC_ATTN_STAGES
+#define KVC_ATTN_STAGES 2
+#endif
+
 constexpr int kThreads = 128;
-constexpr int kTilePages = 4;
-constexpr int kTileRows = kTilePages * kPage;  // 64
 constexpr int kBox = 128;                      // bytes per TMA box row (the swizzle span)
 constexpr float kLn2 = 0.6931471805599453f;
 
+// bf16 pair / fp32 pair of a 32-bit or 64-bit word as a float2
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// 16-byte chunk as float2 pairs
 template <typename T>
-__device__ __forceinline__ void load_chunk(const uint8_t *p, float (&x)[16 / sizeof(T)]);
+__device__ __forceinline__ void load_chunk2(const uint8_t *p, float2 (&x)[16 / sizeof(T) / 2]);
 template <>
-__device__ __forceinline__ void load_chunk<__nv_bfloat16>(const uint8_t *p, float (&x)[8]) {
+__device__ __forceinline__ void load_chunk2<__nv_bfloat16>(const uint8_t *p, float2 (&x)[4]) {
   const uint4 u = *reinterpret_cast<const uint4 *>(p);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[2 * i] = __uint_as_float(w[i] << 16);
-    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
+  x[0] = bf16x2_to_float2(u.x);
+  x[1] = bf16x2_to_float2(u.y);
+  x[2] = bf16x2_to_float2(u.z);
+  x[3] = bf16x2_to_float2(u.w);
 }
 template <>
-__device__ __forceinline__ void load_chunk<float>(const uint8_t *p, float (&x)[4]) {
+__device__ __forceinline__ void load_chunk2<float>(const uint8_t *p, float2 (&x)[2]) {
   const float4 u = *reinterpret_cast<const float4 *>(p);
-  x[0] = u.x;
-  x[1] = u.y;
-  x[2] = u.z;
-  x[3] = u.w;
+  x[0] = make_float2(u.x, u.y);
+  x[1] = make_float2(u.z, u.w);
 }
+// 8 bytes as float2 pairs
 template <typename T>
-__device__ __forceinline__ void load_pair8(const uint8_t *p, float (&x)[8 / sizeof(T)]);
+__device__ __forceinline__ void load_8b2(const uint8_t *p, float2 (&x)[8 / sizeof(T) / 2]);
 template <>
-__device__ __forceinline__ void load_pair8<__nv_bfloat16>(const uint8_t *p, float (&x)[4]) {
+__device__ __forceinline__ void load_8b2<__nv_bfloat16>(const uint8_t *p, float2 (&x)[2]) {
   const uint2 u = *reinterpret_cast<const uint2 *>(p);
-  x[0] = __uint_as_float(u.x << 16);
-  x[1] = __uint_as_float(u.x & 0xffff0000u);
-  x[2] = __uint_as_float(u.y << 16);
-  x[3] = __uint_as_float(u.y & 0xffff0000u);
+  x[0] = bf16x2_to_float2(u.x);
+  x[1] = bf16x2_to_float2(u.y);
 }
 template <>
-__device__ __forceinline__ void load_pair8<float>(const uint8_t *p, float (&x)[2]) {
-  const float2 u = *reinterpret_cast<const float2 *>(p);
-  x[0] = u.x;
-  x[1] = u.y;
+__device__ __forceinline__ void load_8b2<float>(const uint8_t *p, float2 (&x)[1]) {
+  x[0] = *reinterpret_cast<const float2 *>(p);
 }
 __device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
 __device__ __forceinline__ float to_float(float v) { return v; }
@@ -87,42 +90,48 @@ __device__ __forceinline__ float to_float(float v) { return v; }
 template <typename T, int D, int G>
 struct AttnShape {
   static constexpr int kRowBytes = D * (int)sizeof(T);
-  static constexpr int kBoxes = kRowBytes / kBox;           // boxes per row (>= 1)
-  static constexpr int kChunks = kRowBytes / 16;            // 16-byte chunks per row
-  static constexpr int kHalfChunks = kChunks / 2;
-  static constexpr int kEpc = 16 / (int)sizeof(T);          // elements per chunk
-  static constexpr int kPageBox = kPage * kBox;             // 2 KB: one page, one box
-  static constexpr int kPageBytes = kBoxes * kPageBox;      // one page of K (or V)
-  static constexpr int kStageBytes = 2 * kTilePages * kPageBytes;
-  static constexpr int kStages = kStageBytes <= 32768 ? 3 : 2;
-  static constexpr int kVt = 8 / (int)sizeof(T);            // V elements per thread per row
-  static constexpr int kVThreadsPerRow = kRowBytes / 8;
-  static constexpr int kVGroups = kThreads / kVThreadsPerRow;
-  static constexpr int kRedBytes = kVGroups * G * D * 4;
-  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 1024;
-  static_assert(kRowBytes % kBox == 0, "rows must be whole 128-byte boxes");
-  static_assert(kVGroups >= 1 && kThreads % kVThreadsPerRow == 0, "V mapping");
-  static_assert(kRedBytes <= kStages * kStageBytes, "reduction buffer reuses the stages");
+  static constexpr int kBoxes = kRowBytes / kBox;          // 128-byte boxes per row
+  static constexpr int kChunks = kRowBytes / 16;           // 16-byte chunks per row
+  static constexpr int kHalfChunks = kChunks / 2;          // per scoring lane
+  static constexpr int kPairs = 16 / (int)sizeof(T) / 2;   // element pairs per chunk
+  static constexpr int kPageBox = kPage * kBox;            // 2 KB: one page, one box
+  static constexpr int kPageBytes = kBoxes * kPageBox;     // one page of K (or V)
+  static constexpr int kSlotBytes = 2 * kPageBytes;        // K and V of one page
+  static constexpr int kWarpStages = KVC_ATTN_STAGES;      // page slots per warp
+  static constexpr int kWarps = kThreads / 32;
+  static constexpr size_t kSmem = 1024 + (size_t)kWarps * kWarpStages * kSlotBytes;
+  // P.V: each lane owns 8-byte segments of a row; short rows are walked
+  // kRowPar at a time by lane groups
+  static constexpr int kSeg = kRowBytes >= 256 ? kRowBytes / 256 : 1;
+  static constexpr int kRowPar = kRowBytes >= 256 ? 1 : 256 / kRowBytes;
+  static constexpr int kVp = 8 / (int)sizeof(T) / 2;       // element pairs per 8-byte segment
+  static constexpr int kAccPairs = kSeg * kVp;             // accumulator pairs per head per lane
+  static_assert(kRowBytes % kBox == 0 && kRowBytes >= 128 && kRowBytes <= 512, "row size");
+  static_assert((size_t)kWarps * G * D * 4 <= (size_t)kWarps * kWarpStages * kSlotBytes,
+                "the merge buffer reuses the page slots");
 };
 
 // byte offset, inside a page's K (or V) block, of 16-byte chunk c of row rr
-template <int kBoxes>
+// (the 128-byte TMA swizzle: chunk index XOR row index mod 8)
 __device__ __forceinline__ uint32_t chunk_off(int rr, int c) {
   return (uint32_t)((c >> 3) * (kPage * kBox) + rr * kBox + (((c & 7) ^ (rr & 7)) << 4));
 }
 
+// Each of the 4 warps walks every 4th page of the CTA's split through its own
+// 2-slot ring (K and V of one page per slot), with its own running max and
+// sums; no block-wide barrier is taken until the warps' states are merged.
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads) decode_attention_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                    const __grid_constant__ CUtensorMap vmap,
                                                                    DecodeAttnParams p) {
   using S = AttnShape<T, D, G>;
+  constexpr int W = S::kWarps, NS = S::kWarpStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *smem = smem_align<1024>(smem_raw);
   __shared__ __align__(16) float q_s[G][D];
-  __shared__ __align__(16) float p_s[kTileRows][G];
-  __shared__ float wmax[4][G];
-  __shared__ float wsum[4][G];
-  __shared__ __align__(8) uint64_t full[S::kStages];
+  __shared__ __align__(16) float p_s[W][kPage][G];
+  __shared__ float m_s[W][G], l_s[W][G];
+  __shared__ __align__(8) uint64_t full[W][NS];
   __shared__ int abort_flag_s;
   volatile int *abort_flag = &abort_flag_s;
 
@@ -137,195 +146,215 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(const __grid
   const int n_pages = (len + kPage - 1) / kPage;
   const int pg0 = split * p.pages_per_split;
   const int pg1 = min(n_pages, pg0 + p.pages_per_split);
-  const int n_tiles = pg1 > pg0 ? (pg1 - pg0 + kTilePages - 1) / kTilePages : 0;
+  const int n_my = pg1 - pg0 > warp ? (pg1 - pg0 - warp + W - 1) / W : 0;  // pages of this warp
   const int32_t *bt = p.block_table + (int64_t)r * p.bt_stride;
+  uint8_t *ring = smem + warp * NS * S::kSlotBytes;
 
   if (tid == 0) {
-    for (int i = 0; i < S::kStages; ++i) mbar_init(&full[i], 1);
+    for (int w = 0; w < W; ++w)
+      for (int i = 0; i < NS; ++i) mbar_init(&full[w][i], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // this CTA's G query rows, pre-scaled into base 2
-  {
+  {  // this CTA's G query rows, pre-scaled into base 2
     const T *q = reinterpret_cast<const T *>(p.q) + (((int64_t)lc * p.R + r) * p.hq + (int64_t)h * G) * D;
     for (int i = tid; i < G * D; i += kThreads) (&q_s[0][0])[i] = to_float(q[i]) * p.qscale;
   }
   __syncthreads();
 
-  auto issue_tile = [&](int t) {  // one elected thread
-    const int st = t % S::kStages;
-    uint8_t *kd = smem + st * S::kStageBytes;
-    uint8_t *vd = kd + kTilePages * S::kPageBytes;
-    const int a = pg0 + t * kTilePages;
-    const int np = min(kTilePages, pg1 - a);
-    mbar_expect_tx(&full[st], (uint32_t)(np * S::kPageBytes * 2));
-    for (int i = 0; i < np; ++i) {
-      const int64_t row0 = (((int64_t)l * p.num_pages + bt[a + i]) * p.hkv + h) * kPage;
-#pragma unroll
-      for (int b = 0; b < S::kBoxes; ++b) {
-        const int x = b * (kBox / (int)sizeof(T));
-        tma_load_2d(smem_u32(kd + i * S::kPageBytes + b * S::kPageBox), &kmap, x, (int)row0, &full[st]);
-        tma_load_2d(smem_u32(vd + i * S::kPageBytes + b * S::kPageBox), &vmap, x, (int)row0, &full[st]);
-      }
+  // lanes 0 .. 2*kBoxes-1 each issue one box of page k of this warp into its slot
+  auto issue_page = [&](int k) {
+    const int slot = k % NS;
+    const int page = pg0 + warp + k * W;
+    if (lane == 0) mbar_expect_tx(&full[warp][slot], (uint32_t)S::kSlotBytes);
+    __syncwarp();
+    if (lane < 2 * S::kBoxes) {
+      const int b = lane % S::kBoxes;
+      const bool is_v = lane >= S::kBoxes;
+      const int64_t row0 = (((int64_t)l * p.num_pages + bt[page]) * p.hkv + h) * kPage;
+      uint8_t *dst = ring + slot * S::kSlotBytes + (is_v ? S::kPageBytes : 0) + b * S::kPageBox;
+      tma_load_2d(smem_u32(dst), is_v ? &vmap : &kmap, b * (kBox / (int)sizeof(T)), (int)row0,
+                  &full[warp][slot]);
     }
   };
-  if (tid == 0)
-    for (int t = 0; t < min(n_tiles, S::kStages); ++t) issue_tile(t);
+  for (int k = 0; k < min(n_my, NS); ++k) issue_page(k);
 
-  float m_run[G], l_w[G], acc[G][S::kVt];
+  float m_run[G], l_lane[G];
+  float2 acc[G][S::kAccPairs];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     m_run[g] = -INFINITY;
-    l_w[g] = 0.f;
+    l_lane[g] = 0.f;
 #pragma unroll
-    for (int e = 0; e < S::kVt; ++e) acc[g][e] = 0.f;
+    for (int e = 0; e < S::kAccPairs; ++e) acc[g][e] = make_float2(0.f, 0.f);
   }
-  // score mapping: warp w takes page w of the tile; lanes l and l^8 share a row
+  // scoring: lanes l and l^8 share row rr, each takes half of its chunks
   const int half = (lane >> 3) & 1;
   const int rr = (lane & 7) + 8 * (lane >> 4);
-  // V mapping
-  const int vg = tid / S::kVThreadsPerRow;
-  const int vslot = tid % S::kVThreadsPerRow;
+  // P.V: row group and 8-byte segment of this lane
+  const int vgrp = lane / (32 / S::kRowPar);
+  const int vlane = lane % (32 / S::kRowPar);
 
-  int t = 0;
-  for (; t < n_tiles; ++t) {
-    const int st = t % S::kStages;
-    // every thread waits for the tile (acquiring the TMA's writes); the
-    // decision to leave on a timeout is made block-wide below
-    const bool landed = mbar_wait(&full[st], (uint32_t)((t / S::kStages) & 1), abort_flag, p.status);
-    const uint8_t *kt = smem + st * S::kStageBytes;
-    const uint8_t *vt = kt + kTilePages * S::kPageBytes;
-    const int row0 = (pg0 + t * kTilePages) * kPage;  // slot of the tile's first row
-    const int valid = min(kTileRows, len - row0);
+  int k = 0;
+  for (; k < n_my; ++k) {
+    const int slot = k % NS;
+    const bool landed = mbar_wait(&full[warp][slot], (uint32_t)((k / NS) & 1), abort_flag, p.status);
+    if (__any_sync(0xffffffffu, !landed)) break;
+    const uint8_t *kp = ring + slot * S::kSlotBytes;
+    const uint8_t *vp = kp + S::kPageBytes;
+    const int valid = min(kPage, len - (pg0 + warp + k * W) * kPage);
 
-    // 1. scores of row (warp, rr)
-    float s[G];
+    // 1. scores of row rr
+    float2 s2[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) s[g] = 0.f;
-    const uint8_t *kp = kt + warp * S::kPageBytes;
+    for (int g = 0; g < G; ++g) s2[g] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < S::kHalfChunks; ++i) {
       const int c = half * S::kHalfChunks + i;
-      float x[S::kEpc];
-      load_chunk<T>(kp + chunk_off<S::kBoxes>(rr, c), x);
+      float2 x[S::kPairs];
+      load_chunk2<T>(kp + chunk_off(rr, c), x);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
 #pragma unroll
-        for (int e = 0; e < S::kEpc; e += 4) {
-          const float4 qv = *reinterpret_cast<const float4 *>(&q_s[g][c * S::kEpc + e]);
-          s[g] = fmaf(qv.x, x[e], s[g]);
-          s[g] = fmaf(qv.y, x[e + 1], s[g]);
-          s[g] = fmaf(qv.z, x[e + 2], s[g]);
-          s[g] = fmaf(qv.w, x[e + 3], s[g]);
+        for (int e = 0; e < S::kPairs; e += 2) {
+          const float4 qv = *reinterpret_cast<const float4 *>(&q_s[g][(c * S::kPairs + e) * 2]);
+          s2[g] = __ffma2_rn(make_float2(qv.x, qv.y), x[e], s2[g]);
+          s2[g] = __ffma2_rn(make_float2(qv.z, qv.w), x[e + 1], s2[g]);
         }
       }
     }
-    const int row = warp * kPage + rr;
-    const bool ok = row < valid;
+    const bool ok = rr < valid;
+    float pw[G], alpha[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      s[g] += __shfl_xor_sync(0xffffffffu, s[g], 8);
-      s[g] = ok ? s[g] : -INFINITY;
-      float mx = s[g];
+      float sg = s2[g].x + s2[g].y;
+      sg += __shfl_xor_sync(0xffffffffu, sg, 8);
+      sg = ok ? sg : -INFINITY;
+      float mx = sg;
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      if (lane == 0) wmax[warp][g] = mx;
-    }
-    if (__syncthreads_or(!landed)) break;
-    // 2. running max, weights, per-warp sums
-    float alpha[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float tmax = fmaxf(fmaxf(wmax[0][g], wmax[1][g]), fmaxf(wmax[2][g], wmax[3][g]));
-      const float m_new = fmaxf(m_run[g], tmax);
+      const float m_new = fmaxf(m_run[g], mx);  // finite: a page has a valid row
       alpha[g] = exp2f(m_run[g] - m_new);
       m_run[g] = m_new;
-      const float pw = ok ? exp2f(s[g] - m_new) : 0.f;
-      if (half == 0) p_s[row][g] = pw;
-      float sum = half == 0 ? pw : 0.f;
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 8);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 16);
-      l_w[g] = l_w[g] * alpha[g] + sum;
+      pw[g] = ok ? exp2f(sg - m_new) : 0.f;
+      l_lane[g] = fmaf(l_lane[g], alpha[g], half == 0 ? pw[g] : 0.f);
     }
-    __syncthreads();
-    // 3. acc = acc * alpha + P.V over this thread's rows
+    if (half == 0) {
+      if constexpr (G % 4 == 0) {
+#pragma unroll
+        for (int g = 0; g < G; g += 4)
+          *reinterpret_cast<float4 *>(&p_s[warp][rr][g]) = make_float4(pw[g], pw[g + 1], pw[g + 2], pw[g + 3]);
+      } else {
+#pragma unroll
+        for (int g = 0; g < G; ++g) p_s[warp][rr][g] = pw[g];
+      }
+    }
+    __syncwarp();
+    // 2. acc = acc * alpha + P.V over the page's valid rows
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
-      for (int e = 0; e < S::kVt; ++e) acc[g][e] *= alpha[g];
-    {
-      const int c = vslot >> 1;
-      const int sub = (vslot & 1) * 8;
+      for (int e = 0; e < S::kAccPairs; ++e) acc[g][e] = __fmul2_rn(acc[g][e], make_float2(alpha[g], alpha[g]));
 #pragma unroll 4
-      for (int vr = vg; vr < valid; vr += S::kVGroups) {
-        const int pg = vr >> 4, vrr = vr & 15;
-        float x[S::kVt];
-        load_pair8<T>(vt + pg * S::kPageBytes + chunk_off<S::kBoxes>(vrr, c) + sub, x);
-        float pw[G];
-        if constexpr (G % 4 == 0) {
+    for (int vr = vgrp; vr < valid; vr += S::kRowPar) {
+      float w[G];
+      if constexpr (G % 4 == 0) {
 #pragma unroll
-          for (int g = 0; g < G; g += 4) {
-            const float4 w4 = *reinterpret_cast<const float4 *>(&p_s[vr][g]);
-            pw[g] = w4.x;
-            pw[g + 1] = w4.y;
-            pw[g + 2] = w4.z;
-            pw[g + 3] = w4.w;
-          }
-        } else {
-#pragma unroll
-          for (int g = 0; g < G; ++g) pw[g] = p_s[vr][g];
+        for (int g = 0; g < G; g += 4) {
+          const float4 w4 = *reinterpret_cast<const float4 *>(&p_s[warp][vr][g]);
+          w[g] = w4.x;
+          w[g + 1] = w4.y;
+          w[g + 2] = w4.z;
+          w[g + 3] = w4.w;
         }
+      } else {
+#pragma unroll
+        for (int g = 0; g < G; ++g) w[g] = p_s[warp][vr][g];
+      }
+#pragma unroll
+      for (int sg = 0; sg < S::kSeg; ++sg) {
+        const int byte = sg * 256 + vlane * 8;  // 8-byte segment within the row
+        float2 x[S::kVp];
+        load_8b2<T>(vp + chunk_off(vr, byte >> 4) + (byte & 8), x);
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-          for (int e = 0; e < S::kVt; ++e) acc[g][e] = fmaf(pw[g], x[e], acc[g][e]);
+          for (int e = 0; e < S::kVp; ++e)
+            acc[g][sg * S::kVp + e] = __ffma2_rn(make_float2(w[g], w[g]), x[e], acc[g][sg * S::kVp + e]);
       }
     }
-    __syncthreads();  // stage st and p_s are free again
-    if (tid == 0 && t + S::kStages < n_tiles) issue_tile(t + S::kStages);
+    __syncwarp();  // the slot and p_s are free again
+    if (k + NS < n_my) issue_page(k + NS);
   }
-  if (t < n_tiles) {
-    // a wait ran out: let this CTA's copies land (bounded) and leave
-    if (tid == 0)
-      for (int k = t; k < min(n_tiles, t + S::kStages); ++k)
-        mbar_wait(&full[k % S::kStages], (uint32_t)((k / S::kStages) & 1), abort_flag, p.status, false);
-    return;
+  if (k < n_my) {
+    *abort_flag = 1;
+    // let this warp's copies land (bounded) before the CTA may leave
+    if (lane == 0)
+      for (int j = k; j < min(n_my, k + NS); ++j)
+        mbar_wait(&full[warp][j % NS], (uint32_t)((j / NS) & 1), abort_flag, p.status, false);
   }
 
-  // 4. combine the row groups and the warps' sums
-  float *red = reinterpret_cast<float *>(smem);  // [kVGroups][G][D]
-  {
-    const int d0 = vslot * S::kVt;
+  // 3. merge the warps: each writes (max, sum, accumulators)
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float ls = l_lane[g];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    if (lane == 0) {
+      m_s[warp][g] = m_run[g];
+      l_s[warp][g] = ls;
+    }
+  }
+  if constexpr (S::kRowPar > 1) {
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
-      for (int e = 0; e < S::kVt; ++e) red[(vg * G + g) * D + d0 + e] = acc[g][e];
+      for (int e = 0; e < S::kAccPairs; ++e) {
+        acc[g][e].x += __shfl_xor_sync(0xffffffffu, acc[g][e].x, 16);
+        acc[g][e].y += __shfl_xor_sync(0xffffffffu, acc[g][e].y, 16);
+      }
   }
-  if (lane == 0)
+  __syncthreads();  // every warp is past its loop: the page slots are free
+  if (*abort_flag) return;
+  float *red = reinterpret_cast<float *>(smem);  // [W][G][D]
+  if (vgrp == 0) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) wsum[warp][g] = l_w[g];
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int sg = 0; sg < S::kSeg; ++sg) {
+        const int d0 = (sg * 256 + vlane * 8) / (int)sizeof(T);
+#pragma unroll
+        for (int e = 0; e < S::kVp; ++e)
+          *reinterpret_cast<float2 *>(&red[(warp * G + g) * D + d0 + 2 * e]) = acc[g][sg * S::kVp + e];
+      }
+  }
   __syncthreads();
   const int64_t head0 = ((int64_t)lc * p.R + r) * p.hq + (int64_t)h * G;  // first query head row
   for (int i = tid; i < G * D; i += kThreads) {
     const int g = i / D;
-    float o = 0.f;
+    float M = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < S::kVGroups; ++k) o += red[k * G * D + i];
-    const float lsum = wsum[0][g] + wsum[1][g] + wsum[2][g] + wsum[3][g];
+    for (int w = 0; w < W; ++w) M = fmaxf(M, m_s[w][g]);
+    float o = 0.f, lsum = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        if (m_s[w][g] == -INFINITY) continue;
+        const float sc = exp2f(m_s[w][g] - M);
+        o = fmaf(red[(w * G + g) * D + (i % D)], sc, o);
+        lsum = fmaf(l_s[w][g], sc, lsum);
+      }
+    }
     if (p.nsplit == 1) {
       p.out[head0 * D + i] = lsum > 0.f ? o / lsum : 0.f;
-      if (p.lse && (i % D) == 0)
-        p.lse[head0 + g] = lsum > 0.f ? (m_run[g] + log2f(lsum)) * kLn2 : -INFINITY;
+      if (p.lse && (i % D) == 0) p.lse[head0 + g] = lsum > 0.f ? (M + log2f(lsum)) * kLn2 : -INFINITY;
     } else {
       const int64_t pu = (head0 + g) * p.nsplit + split;  // partial row of (query head, split)
       p.part_o[pu * D + (i % D)] = o;
       if ((i % D) == 0) {
-        p.part_ml[pu * 2] = n_tiles > 0 ? m_run[g] : -INFINITY;
+        p.part_ml[pu * 2] = M;
         p.part_ml[pu * 2 + 1] = lsum;
       }
     }

@@ -29,7 +29,7 @@ thread_local std::string g_create_error;
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-  size_t bt, len, prompt, pos, qring, beacons, beacons_s, counts, scores, lse, status, counters,
+  size_t bt, len, prompt, pos, qring, beacons, beacons_s, counts, trig, scores, lse, status, counters,
       stage, attn, total, stage_slot;
 };
 
@@ -84,6 +84,7 @@ Layout make_layout(const kvc_config &c) {
   L.beacons = take(R * Ly * H * B * d * 4);
   L.beacons_s = take(R * Ly * H * B * d * es);
   L.counts = take(R * Ly * H * B * 4);
+  L.trig = take(R * Ly * H * B * 4);
   L.scores = take(B > 0 ? R * Ly * H * (size_t)c.max_seq_len * 4 : 0);
   L.lse = take(R * Ly * H * B * 4);
   L.status = take(256);
@@ -110,7 +111,7 @@ struct kvc_ctx {
   uint8_t *k_pool = nullptr, *v_pool = nullptr, *ws = nullptr;
   int32_t *d_bt = nullptr, *d_len = nullptr, *d_prompt = nullptr, *d_pos = nullptr;
   uint8_t *d_qring = nullptr, *d_beacons_s = nullptr, *d_stage = nullptr;
-  float *d_beacons = nullptr, *d_scores = nullptr, *d_lse = nullptr;
+  float *d_beacons = nullptr, *d_scores = nullptr, *d_lse = nullptr, *d_trig = nullptr;
   int32_t *d_counts = nullptr, *d_status = nullptr;
   unsigned long long *d_counters = nullptr;
   uint8_t *h_stage = nullptr;
@@ -291,6 +292,7 @@ kvc_status kvc_create(const kvc_config *cfg, void *k_pool, void *v_pool, void *w
   c->d_beacons = reinterpret_cast<float *>(c->ws + lay.beacons);
   c->d_beacons_s = c->ws + lay.beacons_s;
   c->d_counts = reinterpret_cast<int32_t *>(c->ws + lay.counts);
+  c->d_trig = reinterpret_cast<float *>(c->ws + lay.trig);
   c->d_scores = reinterpret_cast<float *>(c->ws + lay.scores);
   c->d_lse = reinterpret_cast<float *>(c->ws + lay.lse);
   c->d_status = reinterpret_cast<int32_t *>(c->ws + lay.status);
@@ -512,6 +514,7 @@ kvc_status kvc_update_beacons(kvc_ctx *ctx, int32_t *assign_out, float *ms_out) 
   p.beacons = ctx->d_beacons;
   p.beacons_s = ctx->d_beacons_s;
   p.counts = ctx->d_counts;
+  p.trig = ctx->d_trig;
   p.assign_out = assign_out;
   p.descs = reinterpret_cast<const UpdateDesc *>(st.d);
   p.status = ctx->d_status;
@@ -552,13 +555,15 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
                            kvc_round_stats *stats) {
   if (!ctx) return KVC_ERR_INVALID_ARG;
   const kvc_config &c = ctx->cfg;
-  if (selector != KVC_SEL_RANDOM && selector != KVC_SEL_RANDOM_SHARED && selector != KVC_SEL_BEACON)
+  if (selector != KVC_SEL_RANDOM && selector != KVC_SEL_RANDOM_SHARED && selector != KVC_SEL_BEACON &&
+      selector != KVC_SEL_BEACON_TRIGGER)
     return fail(ctx, KVC_ERR_INVALID_ARG, "unknown selector");
   if (!budgets) return fail(ctx, KVC_ERR_INVALID_ARG, "budgets is NULL");
   const kvc_round_options o = opts ? *opts : kvc_round_options{-1, 1, KVC_COMPACT_ORDERED, 0};
   if (o.block < 1 || o.block > kMaxSeqLen)
     return fail(ctx, KVC_ERR_INVALID_ARG, "block must be in [1, 32768]");
-  if (o.block != 1 && selector == KVC_SEL_BEACON)
+  const bool beacon_sel = selector == KVC_SEL_BEACON || selector == KVC_SEL_BEACON_TRIGGER;
+  if (o.block != 1 && beacon_sel)
     return fail(ctx, KVC_ERR_INVALID_ARG, "block-granular draws apply to the random selectors only");
   if (o.compaction != KVC_COMPACT_ORDERED && o.compaction != KVC_COMPACT_HOLE_FILL)
     return fail(ctx, KVC_ERR_INVALID_ARG, "unknown compaction");
@@ -592,13 +597,13 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
     new_len[r] = P + M;
     new_prompt[r] = P;
     if (M > 0) {
-      if (selector == KVC_SEL_BEACON && !ctx->h_binit[r])
+      if (beacon_sel && !ctx->h_binit[r])
         return fail(ctx, KVC_ERR_STATE, "request " + std::to_string(r) + " has no beacons yet (call kvc_update_beacons)");
       segs.push_back(SegDesc{r, L, P, M});
       tie_by_pos = tie_by_pos || ctx->h_unordered[r];
     }
   }
-  if (selector == KVC_SEL_BEACON && c.num_beacons == 0)
+  if (beacon_sel && c.num_beacons == 0)
     return fail(ctx, KVC_ERR_STATE, "the context has no beacon state (num_beacons = 0)");
   // bucket by candidate count so each launch sizes its shared memory to its segments
   std::stable_sort(segs.begin(), segs.end(), [](const SegDesc &a, const SegDesc &b) {
@@ -618,8 +623,8 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
     KVC_CUDA(ctx, cudaEventRecord(ctx->ev[0], ctx->stream));
   }
   cudaError_t e;
-  float *score_buf = (debug_scores && selector == KVC_SEL_BEACON) ? static_cast<float *>(debug_scores) : ctx->d_scores;
-  if (selector == KVC_SEL_BEACON && !segs.empty()) {
+  float *score_buf = (debug_scores && beacon_sel) ? static_cast<float *>(debug_scores) : ctx->d_scores;
+  if (beacon_sel && !segs.empty()) {
     BeaconScoreParams bp{};
     bp.k_pool = ctx->k_pool;
     bp.block_table = ctx->d_bt;
@@ -627,6 +632,7 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
     bp.beacons_s = ctx->d_beacons_s;
     bp.scores = score_buf;
     bp.lse_out = ctx->d_lse;
+    bp.trig = selector == KVC_SEL_BEACON_TRIGGER ? ctx->d_trig : nullptr;
     bp.status = ctx->d_status;
     bp.num_pages = c.num_pages;
     bp.total_segs = (int64_t)R * per_req_segs;
@@ -654,7 +660,7 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
   sp.pos_map = ctx->d_pos;
   sp.block_table = ctx->d_bt;
   sp.scores = score_buf;
-  sp.debug = (debug_scores && selector != KVC_SEL_BEACON) ? static_cast<uint32_t *>(debug_scores) : nullptr;
+  sp.debug = (debug_scores && !beacon_sel) ? static_cast<uint32_t *>(debug_scores) : nullptr;
   sp.counters = ctx->d_counters;
   sp.status = ctx->d_status;
   sp.num_pages = c.num_pages;
@@ -715,7 +721,7 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
     KVC_CUDA(ctx, cudaMemcpy(&moved, ctx->d_counters, sizeof(moved), cudaMemcpyDeviceToHost));
     st.moved_rows = (int64_t)moved;
     st.compaction_bytes = st.moved_rows * ctx->row_bytes * 2 * 2;
-    if (selector == KVC_SEL_BEACON)
+    if (beacon_sel)
       for (const auto &s : segs) st.key_bytes_scored += (int64_t)s.L * ctx->row_bytes * per_req_segs;
     KVC_CUDA(ctx, cudaEventElapsedTime(&st.ms_score, ctx->ev[0], ctx->ev[1]));
     KVC_CUDA(ctx, cudaEventElapsedTime(&st.ms_select_compact, ctx->ev[1], ctx->ev[2]));
@@ -738,6 +744,7 @@ kvc_status kvc_gather_view(const kvc_ctx *ctx, kvc_view *out) {
   out->beacons = ctx->d_beacons;
   out->beacons_scoring = ctx->d_beacons_s;
   out->beacon_counts = ctx->d_counts;
+  out->beacon_triggers = ctx->d_trig;
   out->max_pages_per_request = ctx->maxp;
   out->row_bytes = ctx->row_bytes;
   out->round = ctx->round;

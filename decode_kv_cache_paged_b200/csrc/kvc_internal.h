@@ -76,6 +76,7 @@ struct BeaconUpdateParams {
   uint8_t *beacons_s;         // scoring copy, dtype
   int32_t *counts;            // [R][layers][Hkv][B]
   int32_t *assign_out;        // optional [R][layers][Hkv][W*G]
+  float *trig;                // [R][layers][Hkv][B]: share of this update's points per beacon
   const UpdateDesc *descs;
   int32_t *status;
   int32_t layers, hkv, hq, G, W, B, d, dtype;
@@ -89,6 +90,7 @@ struct BeaconScoreParams {
   const uint8_t *beacons_s;   // [R][layers][Hkv][B][d] dtype
   float *scores;              // [R][layers][Hkv][max_seq]
   float *lse_out;             // optional [R][layers][Hkv][B]
+  const float *trig;          // cluster-trigger mode: [R][layers][Hkv][B] shares; null = max mode
   int32_t *status;
   int64_t num_pages;
   int64_t total_segs;         // R * layers * Hkv (rows of the beacon arrays / B)

@@ -47,6 +47,9 @@ namespace {
 #ifndef KVC_SC_UNROLL_LARGE
 #define KVC_SC_UNROLL_LARGE 8
 #endif
+#ifndef KVC_SC_UNROLL_HOLE
+#define KVC_SC_UNROLL_HOLE 2
+#endif
 
 // copy / tie variants of the kernel
 constexpr int kOrderedSlotTie = 0;  // order-preserving, ties by slot (slots in position order)
@@ -367,7 +370,9 @@ cudaError_t launch_var(const SelectCompactParams &p, int var, int n_seg_req, int
   switch (var) {
     case kOrderedSlotTie: return launch_one<NT, U, MODE, kOrderedSlotTie>(p, n_seg_req, keys_cap, smem, s);
     case kOrderedPosTie: return launch_one<NT, U, MODE, kOrderedPosTie>(p, n_seg_req, keys_cap, smem, s);
-    default: return launch_one<NT, U, MODE, kHoleFill>(p, n_seg_req, keys_cap, smem, s);
+    // hole filling moves few rows: a short copy chunk keeps registers low and
+    // lets more CTAs per SM hide the latency of the select phase
+    default: return launch_one<NT, KVC_SC_UNROLL_HOLE, MODE, kHoleFill>(p, n_seg_req, keys_cap, smem, s);
   }
 }
 

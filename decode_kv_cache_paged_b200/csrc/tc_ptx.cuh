@@ -15,6 +15,14 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per bounded wait
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+// p rounded up to an A-byte boundary of the shared window (A a power of two),
+// by adding an offset to p itself: the result stays a shared-memory pointer
+// to the compiler, so accesses through it are ld/st.shared, not generic.
+template <uint32_t A, typename T>
+__device__ __forceinline__ T *smem_align(T *p) {
+  uint8_t *b = reinterpret_cast<uint8_t *>(p);
+  return reinterpret_cast<T *>(b + ((A - (smem_u32(b) & (A - 1))) & (A - 1)));
+}
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -82,7 +82,10 @@ typedef enum { KVC_BF16 = 0, KVC_F32 = 1 } kvc_dtype;
 typedef enum {
   KVC_SEL_RANDOM = 0,        /* [RA]: independent Philox score per head and position */
   KVC_SEL_RANDOM_SHARED = 1, /* [RA "发现二"]: one score per (request, layer, position) */
-  KVC_SEL_BEACON = 2         /* [BX]/[BA]: max over beacons of softmax(c.K^T/sqrt(d)) */
+  KVC_SEL_BEACON = 2,        /* [BX]/[BA]: max over beacons of softmax(c.K^T/sqrt(d)) */
+  KVC_SEL_BEACON_TRIGGER = 3 /* [BX] §3.2 cluster-level trigger: sum over beacons of the latest
+                                update's share of points in the beacon's cluster times the
+                                beacon's softmax (see kvc_compress) */
 } kvc_selector;
 
 /* Limits of this build (checked by kvc_create):
@@ -137,6 +140,8 @@ typedef struct {
   float *beacons;             /* [num_requests][num_layers][num_kv_heads][B][head_dim] */
   void *beacons_scoring;      /* same shape, dtype */
   int32_t *beacon_counts;     /* [num_requests][num_layers][num_kv_heads][B] */
+  float *beacon_triggers;     /* [num_requests][num_layers][num_kv_heads][B]: share of the latest
+                                 update's points assigned to each beacon */
   int32_t max_pages_per_request;
   int32_t row_bytes;          /* head_dim * sizeof(dtype) */
   int64_t round;              /* rounds completed */
@@ -218,7 +223,11 @@ kvc_status kvc_update_beacons(kvc_ctx *ctx, int32_t *assign_out, float *ms_out);
  *   Philox4x64-10(counter = (pos, h, l, r), key = (seed, round)); the shared
  *   variant uses h = 2^64-1.  Beacon score (needs initialised beacons) =
  *   max_b exp(z_bj - logsumexp_j' z_bj') with z_bj = c_b.k_j/sqrt(d) over all
- *   cached keys j (prompt included) and c_b the scoring copy.
+ *   cached keys j (prompt included) and c_b the scoring copy.  Cluster-trigger
+ *   score (KVC_SEL_BEACON_TRIGGER; the explainer's "query -> cluster -> KV",
+ *   [BX] §3.2 mark_important, read as: each query of the latest update raises
+ *   the keys its cluster's beacon attends to) = sum_b w_b exp(z_bj - lse_b)
+ *   with w_b the share of the latest update's points assigned to beacon b.
  *   debug_scores: device, NULL or [R][num_layers][num_kv_heads][max_seq_len]
  *     32-bit; receives each candidate's score at index j - P (uint32 for the
  *     random selectors, float for the beacon selector).

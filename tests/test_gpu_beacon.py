@@ -45,7 +45,7 @@ def _fill_recording(ctx, w, gen):
     return qwin
 
 
-def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered"):
+def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered", selector="beacon"):
     ctx = make_context(w)
     if score_impl is not None:
         ctx.set_option(0, score_impl)
@@ -60,6 +60,7 @@ def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered"
     g_beacons = st["beacons"].cpu().numpy().astype(np.float64)
     g_scoring = st["beacons_scoring"].float().cpu().numpy().astype(np.float64)
     g_counts = st["beacon_counts"].cpu().numpy()
+    g_trig = st["beacon_triggers"].cpu().numpy()
     g_assign = assign.cpu().numpy()
     # the scoring copy is the fp32 beacon rounded to the cache dtype (torch's RNE cast)
     assert torch.equal(st["beacons_scoring"], st["beacons"].to(ctx.dtype))
@@ -82,6 +83,9 @@ def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered"
                 near_ties += 1
         c_s, cnt_s, _ = oracle.beacon_update(pts, np.zeros((B, d)), np.zeros(B), init=True, assign_override=ga)
         assert np.array_equal(cnt_s, g_counts[r, l, h])
+        # trigger shares: this update's points per beacon / points (one fp32 division)
+        share = (np.bincount(ga, minlength=B).astype(np.float32) / np.float32(n)).astype(np.float32)
+        assert np.array_equal(g_trig[r, l, h], share), (r, l, h)
         assert np.allclose(g_beacons[r, l, h], c_s, rtol=1e-5, atol=1e-6), (r, l, h)
     # the round
     lengths, prompts = ctx.lengths()
@@ -104,7 +108,7 @@ def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered"
             pre[l] = (full_pos, full_k, full_v)
     scores = torch.zeros((R, Ly, H, ctx.spec.max_seq_len), dtype=torch.float32, device="cuda")
     budgets = w.budget.astype(np.int32)
-    stats = ctx.compress("beacon", budgets, w.philox_seed, debug_scores=scores, stats=True,
+    stats = ctx.compress(selector, budgets, w.philox_seed, debug_scores=scores, stats=True,
                          sink_tokens=sinks, compaction=compaction)
     ctx.sync()
     new_len, _ = ctx.lengths()
@@ -116,7 +120,10 @@ def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered"
         if sinks is not None:
             P = min(P, sinks)
         keys = pre[l][1][r, h, :L].float().cpu().numpy().astype(np.float64)
-        o_sc, _ = oracle.beacon_score(keys, g_scoring[r, l, h], P)
+        if selector == "beacon_trigger":
+            o_sc = oracle.beacon_trigger_score(keys, g_scoring[r, l, h], g_trig[r, l, h].astype(np.float64), P)
+        else:
+            o_sc, _ = oracle.beacon_score(keys, g_scoring[r, l, h], P)
         if L <= K:
             continue
         N, M = L - P, max(0, K - P)
@@ -170,6 +177,22 @@ def test_beacon_round_options(sinks, compaction):
     """Sink-only protection and hole-filling compaction under the beacon selector."""
     out = run_beacon(wl.beacon_serving(R=3, layers=2), sinks=sinks, compaction=compaction)
     print(sinks, compaction, out)
+
+
+@pytest.mark.parametrize("impl", [1, 2], ids=["simt", "tcgen05"])
+def test_cluster_trigger_selector(impl):
+    """The cluster-trigger score (trigger-share-weighted beacon attention) on both kernels."""
+    out = run_beacon(wl.beacon_serving(R=3, layers=2), score_impl=impl, selector="beacon_trigger")
+    print(impl, out)
+
+
+def test_cluster_trigger_256_beacons():
+    w = wl.scaled(wl.long_trace(), num_requests=1, num_layers=2)
+    w.length = np.array([4133])
+    w.budget = np.array([1000])
+    w.prompt = np.array([77])
+    out = run_beacon(w, score_impl=2, selector="beacon_trigger", compaction="hole_fill")
+    print(out)
 
 
 @pytest.mark.parametrize("impl", [1, 2], ids=["simt", "tcgen05"])
