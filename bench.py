@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--requests", type=int, default=None)
     ap.add_argument("--layers", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-pool", action="store_true",
+                    help="also time the oracle over all host cores (one spawned process per core)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--score-impl", type=int, default=0, help="beacon score kernel: 0 auto, 1 SIMT, 2 tcgen05")
@@ -566,7 +568,7 @@ def oracle_attention_rate(w, lengths, budget_s: float):
 
 # ------------------------------------------------------- oracle timing ---
 
-def oracle_sample_rate(w, sel, budget_s: float, rank_seed: int = 0):
+def oracle_sample_rate(w, sel, budget_s: float, rank_seed: int = 0, seg_offset: int = 0):
     """Times the oracle (single thread) on whole segments of the workload until
     ~budget_s seconds of oracle time; returns (head_positions/s, description)."""
     import numpy as np
@@ -580,6 +582,7 @@ def oracle_sample_rate(w, sel, budget_s: float, rank_seed: int = 0):
     n_seg = 0
     H, Ly = w.num_kv_heads, w.num_layers
     segs = [(r, l, h) for r in range(w.num_requests) for l in range(Ly) for h in range(H)]
+    segs = segs[seg_offset % len(segs):] + segs[:seg_offset % len(segs)]
     cache = {}
     while t_total < budget_s and n_seg < len(segs):
         r, l, h = segs[n_seg]
@@ -611,6 +614,38 @@ def oracle_sample_rate(w, sel, budget_s: float, rank_seed: int = 0):
     desc = (f"{n_seg} whole segments (requests from 0, all layers and heads in order) of {w.name}, "
             f"selector {sel}: score + full-sort select + K/V compaction, {t_total:.1f} s of oracle time")
     return hp / t_total, desc, n_seg
+
+
+def _pool_worker(job):
+    """One host core of the all-cores oracle figure (run in a spawned process)."""
+    name, requests, layers, selector, budget_s, offset = job
+    import types
+    args = types.SimpleNamespace(workload=name, requests=requests, layers=layers, selector=selector)
+    w, sel = make_workload(args)
+    t0 = time.perf_counter()
+    rate, _, n_seg = oracle_sample_rate(w, sel, budget_s, rank_seed=offset, seg_offset=offset)
+    return rate * min(budget_s, time.perf_counter() - t0), n_seg, time.perf_counter() - t0
+
+
+def oracle_pool_rate(args, budget_s: float):
+    """The same oracle over all host cores: one single-threaded process per
+    core, each on its own run of whole segments; head-positions/s summed over
+    the processes, divided by the longest process time."""
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+    cores = len(os.sched_getaffinity(0))
+    w, sel = make_workload(args)
+    n_segs = w.num_requests * w.num_layers * w.num_kv_heads
+    jobs = [(args.workload, args.requests, args.layers, sel, budget_s, (i * n_segs) // cores)
+            for i in range(cores)]
+    # spawn (never fork after CUDA is initialised); a worker that dies raises
+    # instead of leaving the pool waiting
+    with ProcessPoolExecutor(max_workers=cores, mp_context=mp.get_context("spawn")) as ex:
+        res = list(ex.map(_pool_worker, jobs, timeout=budget_s * 10 + 120))
+    hp = sum(r[0] for r in res)
+    wall = max(r[2] for r in res)
+    return hp / wall, cores, (f"{sum(r[1] for r in res)} whole segments of {w.name} over {cores} processes "
+                              f"(one per host core), each ~{budget_s:.0f} s of oracle time")
 
 
 def run_reference(args, rank, world):
@@ -689,6 +724,10 @@ def main():
             if not args.no_cpu_baseline:
                 rate, desc, _ = oracle_sample_rate(w, sel, 12.0)
                 out["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+                if args.cpu_pool:
+                    prate, cores, pdesc = oracle_pool_rate(args, 10.0)
+                    out["cpu_baseline_all_cores"] = {"value": prate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                                     "sample": pdesc}
             print(json.dumps(out), flush=True)
     finally:
         if dist:

@@ -257,8 +257,7 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(const __grid
     for (int g = 0; g < G; ++g)
 #pragma unroll
       for (int e = 0; e < S::kAccPairs; ++e) acc[g][e] = __fmul2_rn(acc[g][e], make_float2(alpha[g], alpha[g]));
-#pragma unroll 4
-    for (int vr = vgrp; vr < valid; vr += S::kRowPar) {
+    auto pv_row = [&](int vr) {
       float w[G];
       if constexpr (G % 4 == 0) {
 #pragma unroll
@@ -284,6 +283,14 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(const __grid
           for (int e = 0; e < S::kVp; ++e)
             acc[g][sg * S::kVp + e] = __ffma2_rn(make_float2(w[g], w[g]), x[e], acc[g][sg * S::kVp + e]);
       }
+    };
+    if (valid == kPage) {
+      // full page (all but a segment's last): rows and swizzle offsets known at compile time
+#pragma unroll
+      for (int i = 0; i < kPage / S::kRowPar; ++i) pv_row(i * S::kRowPar + vgrp);
+    } else {
+#pragma unroll 1
+      for (int vr = vgrp; vr < valid; vr += S::kRowPar) pv_row(vr);
     }
     __syncwarp();  // the slot and p_s are free again
     if (k + NS < n_my) issue_page(k + NS);

@@ -166,6 +166,15 @@ def test_beacon_serving_full_size_sampled():
     print(out)
 
 
+@pytest.mark.parametrize("c", [2, 16])
+def test_ragged_beacon_sampled(c):
+    """Ragged lengths 4096..32768 (the ragged sweep's first 4 requests, 2 layers) at 2x and 16x compression,
+    including prompts over budget at 16x: sampled segments."""
+    w = wl.scaled(wl.ragged(c), num_requests=4, num_layers=2)
+    out = run_beacon(w, sample=12)
+    print(c, out)
+
+
 def test_long_trace_sampled():
     w = wl.scaled(wl.long_trace(), num_requests=2, num_layers=4)
     out = run_beacon(w, sample=3)
