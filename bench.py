@@ -490,7 +490,8 @@ def run_attention(args, rank, world, dist):
     alg_bytes = positions * rb * 2 + io_bytes
     mean_ms = statistics.mean(ms)
     roof = {"kernel": "decode_attention", "bound": "hbm", "achieved": alg_bytes / (mean_ms / 1e3) / 1e9,
-            "peak": peaks["hbm_gbs"], "unit": "GB/s", "traffic": None,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "traffic": profiled_traffic("decode_attention", w.name + "/decode_attention", positions),
             "peak_source": f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})",
             "algorithmic_bytes_per_launch": alg_bytes, "launch_ms": mean_ms}
     roof["frac"] = roof["achieved"] / roof["peak"]

@@ -15,24 +15,23 @@
 //   * Work unit = (layer, request, KV head, split of the pages); one CTA of
 //     4 warps each.  Splits give short batches enough CTAs; a second kernel
 //     merges the per-split (max, sum, output) partials.
-//   * Each warp walks every 4th page of the unit on its own: the K and V
-//     rows of a page are 16 consecutive pool rows, fetched as 2-D TMA tiles
-//     (128-byte boxes, 128-byte swizzle, one box per lane) into the warp's
-//     2-slot ring with transaction-count mbarriers.  Warps keep their own
-//     running max and sums, so no block-wide barrier is taken until the
-//     four warps' states are merged at the end.
-//   * Scores: two lanes per row, each half the dimensions; with the swizzle
-//     the 8 lanes of a quarter-warp read 8 rows' chunks from 8 different
-//     bank groups while reading the same query chunk (broadcast).  Online
-//     softmax in base 2 with the scale folded into q.
+//   * Each warp walks every 4th page of the unit on its own: the K rows and
+//     the V rows of a page are each 16 consecutive pool rows, so one bulk
+//     copy apiece (a contiguous 4 KB at bf16 d = 128) brings them into the
+//     warp's 2-slot ring, completing on a transaction-count mbarrier.  Warps
+//     keep their own running max and sums, so no block-wide barrier is taken
+//     until the four warps' states are merged at the end.
+//   * Scores: two lanes per row, each half the dimensions; the 8 lanes of a
+//     quarter-warp take 8 rows and rotate their chunk order by the row, so
+//     their reads of K (256-byte rows) and of the query (48-byte chunk
+//     stride) each fall in 8 different bank groups.  Online softmax in base
+//     2 with the scale folded into q.
 //   * P.V: each lane owns 8-byte segments of a row for all G heads.
 //   * Products and sums use the packed two-wide fp32 FMA of sm_100 (the
 //     same rounding as two scalar FMAs, half the instructions).
 // Every mbarrier wait is bounded: on timeout the kernel records
 // kDevTimeout in the status word, lets its own copies land (bounded) and
 // leaves, all threads of the CTA together.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
 #include "kvc_internal.h"
@@ -46,7 +45,6 @@ namespace {
 #endif
 
 constexpr int kThreads = 128;
-constexpr int kBox = 128;                      // bytes per TMA box row (the swizzle span)
 constexpr float kLn2 = 0.6931471805599453f;
 
 // bf16 pair / fp32 pair of a 32-bit or 64-bit word as a float2
@@ -90,45 +88,40 @@ __device__ __forceinline__ float to_float(float v) { return v; }
 template <typename T, int D, int G>
 struct AttnShape {
   static constexpr int kRowBytes = D * (int)sizeof(T);
-  static constexpr int kBoxes = kRowBytes / kBox;          // 128-byte boxes per row
   static constexpr int kChunks = kRowBytes / 16;           // 16-byte chunks per row
   static constexpr int kHalfChunks = kChunks / 2;          // per scoring lane
   static constexpr int kPairs = 16 / (int)sizeof(T) / 2;   // element pairs per chunk
-  static constexpr int kPageBox = kPage * kBox;            // 2 KB: one page, one box
-  static constexpr int kPageBytes = kBoxes * kPageBox;     // one page of K (or V)
+  static constexpr int kEpc = 2 * kPairs;                  // elements per chunk
+  static constexpr int kQStride = 12;                      // floats per query chunk in shared memory
+  static constexpr int kPageBytes = kPage * kRowBytes;     // one page of K (or V): 16 rows, contiguous
   static constexpr int kSlotBytes = 2 * kPageBytes;        // K and V of one page
   static constexpr int kWarpStages = KVC_ATTN_STAGES;      // page slots per warp
   static constexpr int kWarps = kThreads / 32;
-  static constexpr size_t kSmem = 1024 + (size_t)kWarps * kWarpStages * kSlotBytes;
+  static constexpr size_t kSmem = 128 + (size_t)kWarps * kWarpStages * kSlotBytes;
   // P.V: each lane owns 8-byte segments of a row; short rows are walked
   // kRowPar at a time by lane groups
   static constexpr int kSeg = kRowBytes >= 256 ? kRowBytes / 256 : 1;
   static constexpr int kRowPar = kRowBytes >= 256 ? 1 : 256 / kRowBytes;
   static constexpr int kVp = 8 / (int)sizeof(T) / 2;       // element pairs per 8-byte segment
   static constexpr int kAccPairs = kSeg * kVp;             // accumulator pairs per head per lane
-  static_assert(kRowBytes % kBox == 0 && kRowBytes >= 128 && kRowBytes <= 512, "row size");
+  static_assert(kRowBytes >= 128 && kRowBytes <= 512, "row size");
+  static_assert((kHalfChunks & (kHalfChunks - 1)) == 0, "chunk rotation needs a power of two");
   static_assert((size_t)kWarps * G * D * 4 <= (size_t)kWarps * kWarpStages * kSlotBytes,
                 "the merge buffer reuses the page slots");
 };
-
-// byte offset, inside a page's K (or V) block, of 16-byte chunk c of row rr
-// (the 128-byte TMA swizzle: chunk index XOR row index mod 8)
-__device__ __forceinline__ uint32_t chunk_off(int rr, int c) {
-  return (uint32_t)((c >> 3) * (kPage * kBox) + rr * kBox + (((c & 7) ^ (rr & 7)) << 4));
-}
 
 // Each of the 4 warps walks every 4th page of the CTA's split through its own
 // 2-slot ring (K and V of one page per slot), with its own running max and
 // sums; no block-wide barrier is taken until the warps' states are merged.
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads) decode_attention_kernel(const __grid_constant__ CUtensorMap kmap,
-                                                                   const __grid_constant__ CUtensorMap vmap,
-                                                                   DecodeAttnParams p) {
+__global__ void __launch_bounds__(kThreads) decode_attention_kernel(DecodeAttnParams p) {
   using S = AttnShape<T, D, G>;
   constexpr int W = S::kWarps, NS = S::kWarpStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = smem_align<1024>(smem_raw);
-  __shared__ __align__(16) float q_s[G][D];
+  uint8_t *smem = smem_align<128>(smem_raw);
+  // query chunk c of head g at q_s[g][c]: 48-byte chunk stride, so the 8
+  // lanes of a quarter-warp reading 8 different chunks hit 8 bank groups
+  __shared__ __align__(16) float q_s[G][S::kChunks][S::kQStride];
   __shared__ __align__(16) float p_s[W][kPage][G];
   __shared__ float m_s[W][G], l_s[W][G];
   __shared__ __align__(8) uint64_t full[W][NS];
@@ -158,23 +151,25 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(const __grid
   }
   {  // this CTA's G query rows, pre-scaled into base 2
     const T *q = reinterpret_cast<const T *>(p.q) + (((int64_t)lc * p.R + r) * p.hq + (int64_t)h * G) * D;
-    for (int i = tid; i < G * D; i += kThreads) (&q_s[0][0])[i] = to_float(q[i]) * p.qscale;
+    for (int i = tid; i < G * D; i += kThreads) {
+      const int g = i / D, e = i % D;
+      q_s[g][e / S::kEpc][e % S::kEpc] = to_float(q[i]) * p.qscale;
+    }
   }
   __syncthreads();
 
-  // lanes 0 .. 2*kBoxes-1 each issue one box of page k of this warp into its slot
+  // lanes 0 and 1 copy page k's K and V rows (each one contiguous block of
+  // 16 rows) into the warp's slot
   auto issue_page = [&](int k) {
     const int slot = k % NS;
     const int page = pg0 + warp + k * W;
     if (lane == 0) mbar_expect_tx(&full[warp][slot], (uint32_t)S::kSlotBytes);
     __syncwarp();
-    if (lane < 2 * S::kBoxes) {
-      const int b = lane % S::kBoxes;
-      const bool is_v = lane >= S::kBoxes;
+    if (lane < 2) {
       const int64_t row0 = (((int64_t)l * p.num_pages + bt[page]) * p.hkv + h) * kPage;
-      uint8_t *dst = ring + slot * S::kSlotBytes + (is_v ? S::kPageBytes : 0) + b * S::kPageBox;
-      tma_load_2d(smem_u32(dst), is_v ? &vmap : &kmap, b * (kBox / (int)sizeof(T)), (int)row0,
-                  &full[warp][slot]);
+      const uint8_t *src = (lane ? p.v_pool : p.k_pool) + row0 * S::kRowBytes;
+      bulk_load(smem_u32(ring + slot * S::kSlotBytes + lane * S::kPageBytes), src, (uint32_t)S::kPageBytes,
+                &full[warp][slot]);
     }
   };
   for (int k = 0; k < min(n_my, NS); ++k) issue_page(k);
@@ -210,14 +205,16 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(const __grid
     for (int g = 0; g < G; ++g) s2[g] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < S::kHalfChunks; ++i) {
-      const int c = half * S::kHalfChunks + i;
+      // lanes of a quarter-warp take 8 rows and rotate the chunk order by the
+      // row, so their 16-byte reads fall in 8 different bank groups
+      const int c = half * S::kHalfChunks + ((i + rr) & (S::kHalfChunks - 1));
       float2 x[S::kPairs];
-      load_chunk2<T>(kp + chunk_off(rr, c), x);
+      load_chunk2<T>(kp + rr * S::kRowBytes + c * 16, x);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
 #pragma unroll
         for (int e = 0; e < S::kPairs; e += 2) {
-          const float4 qv = *reinterpret_cast<const float4 *>(&q_s[g][(c * S::kPairs + e) * 2]);
+          const float4 qv = *reinterpret_cast<const float4 *>(&q_s[g][c][2 * e]);
           s2[g] = __ffma2_rn(make_float2(qv.x, qv.y), x[e], s2[g]);
           s2[g] = __ffma2_rn(make_float2(qv.z, qv.w), x[e + 1], s2[g]);
         }
@@ -276,7 +273,7 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(const __grid
       for (int sg = 0; sg < S::kSeg; ++sg) {
         const int byte = sg * 256 + vlane * 8;  // 8-byte segment within the row
         float2 x[S::kVp];
-        load_8b2<T>(vp + chunk_off(vr, byte >> 4) + (byte & 8), x);
+        load_8b2<T>(vp + vr * S::kRowBytes + byte, x);
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
@@ -391,52 +388,23 @@ __global__ void __launch_bounds__(kThreads) decode_attention_merge_kernel(Decode
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void *q = nullptr;
-    cudaDriverEntryPointQueryResult res;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &res) == cudaSuccess &&
-        res == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(q);
-  }
-  return fn;
-}
-
-// pool viewed as [rows][D] of dtype, box (128 bytes of a row, 16 rows), 128-byte swizzle
-bool make_pool_map(CUtensorMap *m, const void *base, uint64_t rows, int D, int dtype) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const int es = dtype == KVC_BF16 ? 2 : 4;
-  cuuint64_t dims[2] = {(cuuint64_t)D, rows};
-  cuuint64_t strides[1] = {(cuuint64_t)D * es};
-  cuuint32_t box[2] = {(cuuint32_t)(kBox / es), (cuuint32_t)kPage};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, dtype == KVC_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-            const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <typename T, int D, int G>
-cudaError_t launch_typed(const CUtensorMap &km, const CUtensorMap &vm, const DecodeAttnParams &p, int units,
-                         cudaStream_t s) {
+cudaError_t launch_typed(const DecodeAttnParams &p, int units, cudaStream_t s) {
   using S = AttnShape<T, D, G>;
   cudaError_t e = cudaFuncSetAttribute(decode_attention_kernel<T, D, G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::kSmem);
   if (e != cudaSuccess) return e;
-  decode_attention_kernel<T, D, G><<<units, kThreads, S::kSmem, s>>>(km, vm, p);
+  decode_attention_kernel<T, D, G><<<units, kThreads, S::kSmem, s>>>(p);
   return cudaGetLastError();
 }
 
 template <typename T, int D>
-cudaError_t launch_g(const CUtensorMap &km, const CUtensorMap &vm, const DecodeAttnParams &p, int G, int units,
-                     cudaStream_t s) {
+cudaError_t launch_g(const DecodeAttnParams &p, int G, int units, cudaStream_t s) {
   switch (G) {
-    case 1: return launch_typed<T, D, 1>(km, vm, p, units, s);
-    case 2: return launch_typed<T, D, 2>(km, vm, p, units, s);
-    case 4: return launch_typed<T, D, 4>(km, vm, p, units, s);
-    default: return launch_typed<T, D, 8>(km, vm, p, units, s);
+    case 1: return launch_typed<T, D, 1>(p, units, s);
+    case 2: return launch_typed<T, D, 2>(p, units, s);
+    case 4: return launch_typed<T, D, 4>(p, units, s);
+    default: return launch_typed<T, D, 8>(p, units, s);
   }
 }
 
@@ -444,25 +412,19 @@ cudaError_t launch_g(const CUtensorMap &km, const CUtensorMap &vm, const DecodeA
 
 bool decode_attention_supported(int dtype, int head_dim, int G) {
   return (dtype == KVC_BF16 || dtype == KVC_F32) && (head_dim == 64 || head_dim == 128) &&
-         (G == 1 || G == 2 || G == 4 || G == 8) && encode_fn() != nullptr;
+         (G == 1 || G == 2 || G == 4 || G == 8);
 }
 
-cudaError_t launch_decode_attention(const DecodeAttnParams &p, const void *k_pool, const void *v_pool,
-                                    int64_t pool_rows, int head_dim, int dtype, int G, int *launches,
+cudaError_t launch_decode_attention(const DecodeAttnParams &p, int head_dim, int dtype, int G, int *launches,
                                     cudaStream_t s) {
   *launches = 0;
-  CUtensorMap km, vm;
-  if (!make_pool_map(&km, k_pool, (uint64_t)pool_rows, head_dim, dtype) ||
-      !make_pool_map(&vm, v_pool, (uint64_t)pool_rows, head_dim, dtype))
-    return cudaErrorInvalidValue;
   const int units = p.layer_count * p.R * p.hkv * p.nsplit;
   if (units <= 0) return cudaSuccess;
   cudaError_t e;
   if (dtype == KVC_BF16)
-    e = head_dim == 128 ? launch_g<__nv_bfloat16, 128>(km, vm, p, G, units, s)
-                        : launch_g<__nv_bfloat16, 64>(km, vm, p, G, units, s);
+    e = head_dim == 128 ? launch_g<__nv_bfloat16, 128>(p, G, units, s) : launch_g<__nv_bfloat16, 64>(p, G, units, s);
   else
-    e = head_dim == 128 ? launch_g<float, 128>(km, vm, p, G, units, s) : launch_g<float, 64>(km, vm, p, G, units, s);
+    e = head_dim == 128 ? launch_g<float, 128>(p, G, units, s) : launch_g<float, 64>(p, G, units, s);
   if (e != cudaSuccess) return e;
   *launches = 1;
   if (p.nsplit > 1) {

@@ -795,11 +795,9 @@ kvc_status kvc_decode_attention(kvc_ctx *ctx, int32_t layer_begin, int32_t layer
   if (((uintptr_t)q % ctx->es) || ((uintptr_t)out & 3) || ((uintptr_t)lse & 3))
     return fail(ctx, KVC_ERR_INVALID_ARG, "q, out or lse misaligned");
   const int G = ctx->G;
-  const int64_t pool_rows = (int64_t)c.num_layers * c.num_pages * c.num_kv_heads * kPage;
-  if (!decode_attention_supported(c.dtype, c.head_dim, G) || pool_rows >= ((int64_t)1 << 31))
+  if (!decode_attention_supported(c.dtype, c.head_dim, G))
     return fail(ctx, KVC_ERR_UNSUPPORTED,
-                "decode attention needs bf16 or f32, head_dim 64 or 128, 1, 2, 4 or 8 query heads per KV "
-                "head and fewer than 2^31 pool rows");
+                "decode attention needs bf16 or f32, head_dim 64 or 128 and 1, 2, 4 or 8 query heads per KV head");
   const int R = c.num_requests;
   int max_len = 0;
   for (int r = 0; r < R; ++r) max_len = std::max(max_len, ctx->h_len[r]);
@@ -816,6 +814,8 @@ kvc_status kvc_decode_attention(kvc_ctx *ctx, int32_t layer_begin, int32_t layer
   pps = (pps + 3) & ~3;
   nsplit = std::max(1, (np_max + pps - 1) / pps);
   DecodeAttnParams p{};
+  p.k_pool = ctx->k_pool;
+  p.v_pool = ctx->v_pool;
   p.q = static_cast<const uint8_t *>(q);
   p.block_table = ctx->d_bt;
   p.lengths = ctx->d_len;
@@ -836,8 +836,7 @@ kvc_status kvc_decode_attention(kvc_ctx *ctx, int32_t layer_begin, int32_t layer
   p.qscale = (scale > 0.f ? scale : 1.0f / std::sqrt((float)c.head_dim)) * 1.4426950408889634f;
   if (ms_out) KVC_CUDA(ctx, cudaEventRecord(ctx->ev[0], ctx->stream));
   int launches = 0;
-  cudaError_t e = launch_decode_attention(p, ctx->k_pool, ctx->v_pool, pool_rows, c.head_dim, c.dtype, G,
-                                          &launches, ctx->stream);
+  cudaError_t e = launch_decode_attention(p, c.head_dim, c.dtype, G, &launches, ctx->stream);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "decode_attention");
   if (ms_out) {
     KVC_CUDA(ctx, cudaEventRecord(ctx->ev[1], ctx->stream));

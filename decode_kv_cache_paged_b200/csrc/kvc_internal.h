@@ -52,6 +52,7 @@ constexpr int kScHoleFill = 2;  // hole-filling compaction (implies ties by posi
 
 // One decode step of attention over the cache (decode_attention.cu).
 struct DecodeAttnParams {
+  const uint8_t *k_pool, *v_pool;  // [layers][pages][Hkv][16][d] dtype
   const uint8_t *q;            // [layer_count][R][Hq][d] dtype
   const int32_t *block_table;  // [R][bt_stride]
   const int32_t *lengths;      // [R] device lengths
@@ -114,8 +115,7 @@ cudaError_t launch_gather_dense(const uint8_t *k_pool, const uint8_t *v_pool,
                                 int cap, int hkv, int row_bytes, int64_t num_pages, int bt_stride,
                                 uint8_t *k_out, uint8_t *v_out, int32_t *pos_out, cudaStream_t s);
 bool decode_attention_supported(int dtype, int head_dim, int G);
-cudaError_t launch_decode_attention(const DecodeAttnParams &p, const void *k_pool, const void *v_pool,
-                                    int64_t pool_rows, int head_dim, int dtype, int G, int *launches,
+cudaError_t launch_decode_attention(const DecodeAttnParams &p, int head_dim, int dtype, int G, int *launches,
                                     cudaStream_t s);
 cudaError_t launch_select_compact(const SelectCompactParams &p, int mode, int n_seg_req,
                                   int max_n, int max_m, cudaStream_t s);
