@@ -52,18 +52,11 @@ namespace kvc {
 namespace {
 
 constexpr int kTileKeys = 128;
-#ifndef KVC_TC_CPASYNC
-#define KVC_TC_CPASYNC 0
-#endif
-// Key tiles arrive either as 2-D TMA boxes (one arrival with the byte count)
-// or as the producer warp's cp.async copies (one arrival per lane).
-constexpr uint32_t kKeyArrivals = KVC_TC_CPASYNC ? 32u : 1u;
 constexpr int kEpiWarps = 8;   // two groups of 4: group g drains accumulator buffer g
 constexpr int kThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr uint32_t kTmemCols = 512;
 
 struct TcParams {
-  const uint8_t *k_pool;  // [layers][pages][Hkv][16][128] bf16
   const int32_t *block_table;
   const SegDesc *segs;
   float *scores;
@@ -133,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], kKeyArrivals);
+      mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -168,7 +161,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // results and the abort flag broadcast); lane q issues the two loads of
     // page q of each tile, so a tile's 16 loads leave in one instruction.
     constexpr int kTP = kTileKeys / kPage;
-    const uint8_t *k_bytes = p.k_pool;
     auto uniform_abort = [&]() { return __shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0) != 0; };
     uint32_t it = 0;  // key-tile counter across segments
     int si = 0;       // local segment counter
@@ -206,29 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (t >= g.n1 && t - g.n1 < g.nres) {
-          // the tile is still in this stage from pass 1
-          if (kKeyArrivals == 32 || lane == 0) mbar_arrive(&full[st]);
-        } else if (kKeyArrivals == 32) {
-          // 128 key rows x 16 chunks of 16 bytes: lane handles chunk (lane & 15)
-          // of two rows per page, written straight into the swizzled layout;
-          // rows of pages past the segment are zero-filled
-          uint8_t *dst = kbuf + st * kTileBytes;
-          const int c = lane & 15;
-#pragma unroll
-          for (int q = 0; q < kTP; ++q) {
-            const int pg_q = __shfl_sync(0xffffffffu, pg_cur, q);
-            const bool have = tile * kTP + q < pages;
-            const uint8_t *page_src =
-                k_bytes + ((((int64_t)g.l * p.num_pages + pg_q) * p.hkv + g.h) * kPage) * 256 + c * 16;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int rip = 2 * i + (lane >> 4);  // row within the page
-              const int row = q * kPage + rip;
-              cp_async16(smem_u32(dst + (c >> 3) * (kTileKeys * 128) + row * 128 + (((c & 7) ^ (row & 7)) << 4)),
-                         have ? page_src + rip * 256 : k_bytes, have ? 16u : 0u);
-            }
-          }
-          cp_async_arrive(&full[st]);
+          if (lane == 0) mbar_arrive(&full[st]);  // the tile is still in this stage from pass 1
         } else {
           const int npg = min(kTP, pages - tile * kTP);
           if (lane == 0) mbar_expect_tx(&full[st], (uint32_t)npg * 2u * 2048u);
@@ -245,7 +215,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
-    if (kKeyArrivals == 32) asm volatile("cp.async.wait_all;" ::: "memory");
     if (lane == 0 && *abort_flag) {
       // let loads already issued land before the CTA's shared memory goes away
       for (int i = 0; i < kStages && it > 0; ++i) {
@@ -273,8 +242,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&full[st], (it / kStages) & 1, abort_flag, p.status) &&
                mbar_wait(&acc_empty[buf], ((acc_it >> 1) & 1) ^ 1, abort_flag, p.status);
           if (!ok) break;
-          // key rows written by cp.async (generic proxy) are read by the MMA
-          if (kKeyArrivals == 32) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           tmem_fence_after();
           const uint32_t k_addr = smem_u32(kbuf + st * kTileBytes);
           const uint32_t d = tmem_base + buf * 256;
@@ -525,7 +492,6 @@ cudaError_t launch_beacon_score_tc(const BeaconScoreParams &p, int n_req, int ma
   if (!make_map(&km, p.k_pool, krows, kPage) || !make_map(&cm, p.beacons_s, crows, (uint32_t)p.B))
     return cudaErrorInvalidValue;
   TcParams tp{};
-  tp.k_pool = p.k_pool;
   tp.block_table = p.block_table;
   tp.segs = p.segs;
   tp.scores = p.scores;

@@ -63,11 +63,16 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
 
 // k_in-th largest key (1-based) among the candidates for which keyfn(j, key)
 // returns true; also how many keys equal it (count_eq) and how many of those
-// belong to the top k_in (need).
+// belong to the top k_in (need).  MSB radix select with 8-bit digits; once
+// the bucket holding the answer has at most kFinish keys (for random 32-bit
+// keys that is after the first digit), those keys are gathered and one warp
+// finishes by counting, so the remaining passes over all keys are skipped.
+constexpr int kFinish = 64;
+
 template <int NT, class KeyFn>
 __device__ __forceinline__ void block_radix_select(int n, int k_in, KeyFn keyfn, uint32_t *hist,
-                                                   uint32_t *bcast, uint32_t &tau, int &need,
-                                                   int &count_eq) {
+                                                   uint32_t *bcast, uint32_t *cand, uint32_t &tau,
+                                                   int &need, int &count_eq) {
   uint32_t prefix = 0, mask = 0;
   int k = k_in;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -114,6 +119,7 @@ __device__ __forceinline__ void block_radix_select(int n, int k_in, KeyFn keyfn,
         bcast[0] = (uint32_t)digit;
         bcast[1] = (uint32_t)k - cum;
         bcast[2] = cnt;
+        bcast[3] = 0;
       }
     }
     __syncthreads();
@@ -121,38 +127,85 @@ __device__ __forceinline__ void block_radix_select(int n, int k_in, KeyFn keyfn,
     mask |= 255u << shift;
     k = (int)bcast[1];
     count_eq = (int)bcast[2];
+    if (shift > 0 && count_eq <= kFinish) {
+      // gather the bucket, then one warp counts: the k-th largest x has
+      // #{y > x} < k <= #{y >= x}
+      for (int j = tid; j < n; j += NT) {
+        uint32_t key;
+        if (keyfn(j, key) && (key & mask) == prefix) cand[atomicAdd(&bcast[3], 1u)] = key;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const int m = count_eq;
+#pragma unroll
+        for (int h = 0; h < kFinish / 32; ++h) {
+          const int i = h * 32 + lane;
+          if (i < m) {
+            const uint32_t x = cand[i];
+            int gt = 0, ge = 0;
+            for (int t = 0; t < m; ++t) {
+              const uint32_t y = cand[t];
+              gt += y > x;
+              ge += y >= x;
+            }
+            if (gt < k && k <= ge) {  // every lane holding the answer writes the same values
+              bcast[0] = x;
+              bcast[1] = (uint32_t)(k - gt);
+              bcast[2] = (uint32_t)(ge - gt);
+            }
+          }
+        }
+      }
+      __syncthreads();
+      tau = bcast[0];
+      need = (int)bcast[1];
+      count_eq = (int)bcast[2];
+      __syncthreads();  // bcast and cand are reused by the caller's next select
+      return;
+    }
     __syncthreads();
   }
   tau = prefix;
   need = k;
 }
 
-// Tile-wise exclusive scan of a per-candidate predicate over [lo, hi) in
-// candidate order; calls fn(j, index) for every j with pred(j) true, index =
-// number of earlier candidates with pred true.  Returns the total.
+// Exclusive scan of a per-candidate predicate over [lo, hi) in candidate
+// order; calls fn(j, index) for every j with pred(j) true, index = number of
+// earlier candidates with pred true.  Returns the total.  Each warp owns a
+// contiguous range (whole 32-candidate chunks): it counts its range with
+// ballots, one block barrier exchanges the warp totals, and a second sweep
+// hands out the indices, so the block synchronises once per scan instead of
+// once per chunk.
 template <int NT, class Pred, class Fn>
 __device__ __forceinline__ int block_scan_each(int lo, int hi, Pred pred, Fn fn, uint32_t *warp_cnt) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int carry = 0;
-#pragma unroll 1
-  for (int base = lo; base < hi; base += NT) {
-    const int j = base + tid;
-    const bool f = j < hi && pred(j);
-    const unsigned m = __ballot_sync(0xffffffffu, f);
-    if (lane == 0) warp_cnt[warp] = __popc(m);
-    __syncthreads();
-    int off = carry, tot = 0;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w) {
-      const int c = warp_cnt[w];
-      if (w < warp) off += c;
-      tot += c;
-    }
-    if (f) fn(j, off + __popc(m & ((1u << lane) - 1u)));
-    carry += tot;
-    __syncthreads();  // warp_cnt reuse
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = hi - lo;
+  const int per = ((n + NW * 32 - 1) / (NW * 32)) * 32;  // candidates per warp
+  const int w0 = lo + warp * per, w1 = min(hi, w0 + per);
+  int cnt = 0;
+  for (int base = w0; base < w1; base += 32) {
+    const int j = base + lane;
+    cnt += __popc(__ballot_sync(0xffffffffu, j < w1 && pred(j)));
   }
-  return carry;
+  if (lane == 0) warp_cnt[warp] = cnt;
+  __syncthreads();
+  int off = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const int c = warp_cnt[w];
+    if (w < warp) off += c;
+    tot += c;
+  }
+  for (int base = w0; base < w1; base += 32) {
+    const int j = base + lane;
+    const bool f = j < w1 && pred(j);
+    const unsigned m = __ballot_sync(0xffffffffu, f);
+    if (f) fn(j, off + __popc(m & ((1u << lane) - 1u)));
+    off += __popc(m);
+  }
+  __syncthreads();  // warp_cnt reuse
+  return tot;
 }
 
 template <int NT, int MODE, int kUnroll, int VAR>
@@ -161,7 +214,8 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
   uint32_t *keys = reinterpret_cast<uint32_t *>(smem);                  // [keys_cap]
   uint16_t *src_of_rank = reinterpret_cast<uint16_t *>(keys + keys_cap);  // [keys_cap]
   __shared__ uint32_t hist[256];
-  __shared__ uint32_t bcast[3];
+  __shared__ uint32_t bcast[4];
+  __shared__ uint32_t cand[kFinish];
   __shared__ uint32_t warp_cnt[NT / 32], warp_eq[NT / 32];
   __shared__ int first_evicted;
 
@@ -200,7 +254,7 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
   uint32_t tau;
   int need, count_eq;
   block_radix_select<NT>(
-      N, M, [&](int j, uint32_t &k) { k = keys[j]; return true; }, hist, bcast, tau, need, count_eq);
+      N, M, [&](int j, uint32_t &k) { k = keys[j]; return true; }, hist, bcast, cand, tau, need, count_eq);
   // with ties split and slots possibly out of position order: the `need`
   // lowest positions among the tied keys (positions are distinct)
   uint32_t ptau = 0;
@@ -214,7 +268,7 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
           k = ~(uint32_t)p.pos_map[row_of(P + j)];
           return true;
         },
-        hist, bcast, ptau, need2, cnt2);
+        hist, bcast, cand, ptau, need2, cnt2);
   }
   auto kept_pos = [&](int j) -> bool {  // kept flag when ties go by position
     const uint32_t key = keys[j];
@@ -232,34 +286,40 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
   if (VAR != kHoleFill) {
     // 3. ranks in slot order
     if (VAR == kOrderedSlotTie) {
-      // kept = key > tau, or key == tau among the first `need` such slots
-      int carry_gt = 0, carry_eq = 0;
-#pragma unroll 1
-      for (int base = 0; base < N; base += NT) {
-        const int j = base + tid;
-        const bool valid = j < N;
+      // kept = key > tau, or key == tau among the first `need` such slots:
+      // two counts per candidate (greater, equal) scanned over warp ranges
+      constexpr int NW = NT / 32;
+      const int per = ((N + NW * 32 - 1) / (NW * 32)) * 32;
+      const int w0 = warp * per, w1 = min(N, w0 + per);
+      int cgt = 0, ceq = 0;
+      for (int base = w0; base < w1; base += 32) {
+        const int j = base + lane;
+        const uint32_t key = j < w1 ? keys[j] : 0u;
+        cgt += __popc(__ballot_sync(0xffffffffu, j < w1 && key > tau));
+        ceq += __popc(__ballot_sync(0xffffffffu, j < w1 && key == tau));
+      }
+      if (lane == 0) {
+        warp_cnt[warp] = cgt;
+        warp_eq[warp] = ceq;
+      }
+      __syncthreads();
+      int off_gt = 0, off_eq = 0;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        if (w < warp) {
+          off_gt += warp_cnt[w];
+          off_eq += warp_eq[w];
+        }
+      }
+      const unsigned lt_mask = (1u << lane) - 1u;
+      for (int base = w0; base < w1; base += 32) {
+        const int j = base + lane;
+        const bool valid = j < w1;
         const uint32_t key = valid ? keys[j] : 0u;
         const bool gt = valid && key > tau;
         const bool eq = valid && key == tau;
         const unsigned mgt = __ballot_sync(0xffffffffu, gt);
         const unsigned meq = __ballot_sync(0xffffffffu, eq);
-        const unsigned lt_mask = (1u << lane) - 1u;
-        if (lane == 0) {
-          warp_cnt[warp] = __popc(mgt);
-          warp_eq[warp] = __popc(meq);
-        }
-        __syncthreads();
-        int off_gt = carry_gt, off_eq = carry_eq, tot_gt = 0, tot_eq = 0;
-#pragma unroll
-        for (int w = 0; w < NT / 32; ++w) {
-          const int g = warp_cnt[w], e = warp_eq[w];
-          if (w < warp) {
-            off_gt += g;
-            off_eq += e;
-          }
-          tot_gt += g;
-          tot_eq += e;
-        }
         const int gt_before = off_gt + __popc(mgt & lt_mask);
         const int eq_before = off_eq + __popc(meq & lt_mask);
         const bool kept = gt || (eq && eq_before < need);
@@ -268,9 +328,8 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
         } else if (valid) {
           atomicMin(&first_evicted, j);
         }
-        carry_gt += tot_gt;
-        carry_eq += tot_eq;
-        __syncthreads();
+        off_gt += __popc(mgt);
+        off_eq += __popc(meq);
       }
     } else {
       block_scan_each<NT>(

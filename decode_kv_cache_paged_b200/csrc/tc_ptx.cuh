@@ -85,15 +85,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
-// 16-byte cp.async (L2 only); src_bytes 0 zero-fills the destination.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-// One arrival on `bar` once all of this thread's earlier cp.async copies have
-// landed (the barrier's expected count includes it).
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 // Bulk copy of `bytes` contiguous bytes (both addresses 16-byte aligned, a
 // multiple of 16 bytes) into this CTA's shared memory, completing as
 // transaction bytes on `bar`.  No multicast.
