@@ -94,6 +94,22 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
                  "r"(tmem_cols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  // this thread's point of the next tile, loaded into registers one tile
+  // ahead (the first before the beacon preparation) so the global latency
+  // overlaps the work on the current tile
+  uint4 xw[16];
+  auto load_point = [&](int p0) {
+    const int pt = p0 + tid;
+    if (pt < n_pts) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(ring + point_base(pt));
+#pragma unroll
+      for (int c = 0; c < 16; ++c) xw[c] = src[c];
+    } else {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) xw[c] = make_uint4(0, 0, 0, 0);
+    }
+  };
+  load_point(0);
   // the one-hot tile starts at zero; counts at zero
   for (int i = tid; i < 32768 / 16; i += kUT) reinterpret_cast<uint4 *>(asum)[i] = make_uint4(0, 0, 0, 0);
   for (int b = tid; b < B; b += kUT) cnt[b] = 0;
@@ -139,20 +155,10 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
   int phase = 0;
   for (int p0 = 0; p0 < n_pts; p0 += 128) {
     const int pt = p0 + tid;
-    if (pt < n_pts) {
-      const uint4 *src = reinterpret_cast<const uint4 *>(ring + point_base(pt));
-      uint4 w[16];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) w[c] = src[c];
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        *reinterpret_cast<uint4 *>(xs + (c >> 3) * 16384 + tid * 128 + (((c & 7) ^ (tid & 7)) << 4)) = w[c];
-    } else {
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        *reinterpret_cast<uint4 *>(xs + (c >> 3) * 16384 + tid * 128 + (((c & 7) ^ (tid & 7)) << 4)) =
-            make_uint4(0, 0, 0, 0);
-    }
+    for (int c = 0; c < 16; ++c)
+      *reinterpret_cast<uint4 *>(xs + (c >> 3) * 16384 + tid * 128 + (((c & 7) ^ (tid & 7)) << 4)) = xw[c];
+    if (p0 + 128 < n_pts) load_point(p0 + 128);  // in flight during this tile
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tmem_fence_before();
     __syncthreads();
@@ -238,22 +244,33 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
       float4 *g4 = reinterpret_cast<float4 *>(gbeac + (int64_t)b * D);
       __nv_bfloat162 *s2 = reinterpret_cast<__nv_bfloat162 *>(reinterpret_cast<__nv_bfloat16 *>(p.beacons_s) +
                                                                (seg * B + b) * D);
+      // old values of 32 dimensions, the next chunk's loads in flight while
+      // this chunk is combined and stored
+      float4 ov[8];
+      auto load_old = [&](int c0) {
+        if (mine && !ud.init)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) ov[q] = g4[c0 / 4 + q];
+      };
+      load_old(0);
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         float sm[32];
         tmem_ld32(tmem_base + lane_addr + acol + 128u * hh + c0, sm);  // warp-collective
+        float v[32];
         if (mine) {
-          float v[32];
           if (ud.init) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = c_old(b, c0 + i);
           } else {
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-              const float4 o = g4[c0 / 4 + q];
-              v[4 * q] = o.x; v[4 * q + 1] = o.y; v[4 * q + 2] = o.z; v[4 * q + 3] = o.w;
+              v[4 * q] = ov[q].x; v[4 * q + 1] = ov[q].y; v[4 * q + 2] = ov[q].z; v[4 * q + 3] = ov[q].w;
             }
           }
+        }
+        if (c0 + 32 < D) load_old(c0 + 32);
+        if (mine) {
           if (m > 0)
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = ((float)n * v[i] + sm[i]) / (float)(n + m);
