@@ -114,6 +114,7 @@ _SIGS = {
     "kvc_gather_view": (_i32, [_P, ctypes.POINTER(kvc_view)]),
     "kvc_get_lengths": (_i32, [_P, _P, _P]),
     "kvc_gather_dense": (_i32, [_P, _i32, _i32, _i32, _i32, _P, _P, _P]),
+    "kvc_check_wait_timeout": (_i32, [_P, ctypes.c_uint32]),
     "kvc_sync": (_i32, [_P]),
     "kvc_status_string": (ctypes.c_char_p, [_i32]),
     "kvc_last_error": (ctypes.c_char_p, [_P]),
@@ -270,6 +271,11 @@ class Context:
         _check(kvc_decode_attention(self.handle, int(layer_begin), int(lc), _ptr(q), ctypes.c_float(scale),
                                     _ptr(out), _ptr(lse), ctypes.byref(ms) if timed else None), self.handle)
         return (out, lse, ms.value) if timed else (out, lse)
+
+    def check_wait_timeout(self, limit_ms: int = 100):
+        """kvc_check_wait_timeout: raises KvcError(KVC_ERR_DEVICE_TIMEOUT) when the
+        bounded-wait failure detection works."""
+        _check(kvc_check_wait_timeout(self.handle, int(limit_ms)), self.handle)
 
     def sync(self):
         _check(kvc_sync(self.handle), self.handle)

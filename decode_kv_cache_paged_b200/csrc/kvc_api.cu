@@ -847,6 +847,16 @@ kvc_status kvc_decode_attention(kvc_ctx *ctx, int32_t layer_begin, int32_t layer
   return KVC_OK;
 }
 
+kvc_status kvc_check_wait_timeout(kvc_ctx *ctx, uint32_t limit_ms) {
+  if (!ctx) return KVC_ERR_INVALID_ARG;
+  if (limit_ms < 1 || limit_ms > 2000) return fail(ctx, KVC_ERR_INVALID_ARG, "limit_ms must be in [1, 2000]");
+  KVC_CUDA(ctx, cudaSetDevice(ctx->device));
+  if (kvc_status st = take_device_status(ctx)) return st;  // an earlier error is reported as such
+  cudaError_t e = launch_wait_timeout_probe(ctx->d_status, limit_ms, ctx->stream);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "wait_timeout_probe");
+  return take_device_status(ctx);
+}
+
 kvc_status kvc_sync(kvc_ctx *ctx) {
   if (!ctx) return KVC_ERR_INVALID_ARG;
   KVC_CUDA(ctx, cudaSetDevice(ctx->device));

@@ -114,6 +114,7 @@ cudaError_t launch_gather_dense(const uint8_t *k_pool, const uint8_t *v_pool,
                                 const int32_t *lengths, int layer, int req_begin, int req_count,
                                 int cap, int hkv, int row_bytes, int64_t num_pages, int bt_stride,
                                 uint8_t *k_out, uint8_t *v_out, int32_t *pos_out, cudaStream_t s);
+cudaError_t launch_wait_timeout_probe(int32_t *status, uint32_t limit_ms, cudaStream_t s);
 bool decode_attention_supported(int dtype, int head_dim, int G);
 cudaError_t launch_decode_attention(const DecodeAttnParams &p, int head_dim, int dtype, int G, int *launches,
                                     cudaStream_t s);

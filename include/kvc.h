@@ -311,6 +311,17 @@ kvc_status kvc_get_lengths(const kvc_ctx *ctx, int32_t *lengths, int32_t *prompt
 kvc_status kvc_gather_dense(kvc_ctx *ctx, int32_t layer, int32_t req_begin, int32_t req_count,
                             int32_t cap, void *k_out, void *v_out, int32_t *pos_out);
 
+/* Failure-detection self-test (no counterpart in the pages).  Every wait of
+ * the library's kernels on a device-side event is bounded; when the bound
+ * runs out the kernel records a timeout in the status word and returns,
+ * leaving the context usable, and the next synchronising call returns
+ * KVC_ERR_DEVICE_TIMEOUT.  This call exercises that path: it enqueues a
+ * one-thread kernel that waits, with a bound of limit_ms (1..2000), on an
+ * mbarrier nothing arrives on, synchronises, and returns
+ * KVC_ERR_DEVICE_TIMEOUT (status cleared) when detection works.  A device
+ * error latched before the call is returned first, as itself. */
+kvc_status kvc_check_wait_timeout(kvc_ctx *ctx, uint32_t limit_ms);
+
 /* Waits for the stream and reports any latched device error (then clears it). */
 kvc_status kvc_sync(kvc_ctx *ctx);
 

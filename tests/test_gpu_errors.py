@@ -1,6 +1,7 @@
 """Error paths of the ABI on a GPU.  Every failure is made on the host (bad
 arguments, exhausted pools, wrong call order, a NaN planted in the input
-queries); none faults, traps or hangs the device."""
+queries) or is a bounded device wait that runs out by design; none faults,
+traps or hangs the device."""
 import ctypes
 
 import numpy as np
@@ -128,3 +129,20 @@ def test_host_pinned_append_matches_device_append():
     assert torch.equal(a.state_tensors()["query_ring"], b.state_tensors()["query_ring"])
     a.close()
     b.close()
+
+
+def test_bounded_wait_timeout_is_reported_and_the_context_survives():
+    """A device wait that runs out (an mbarrier nothing arrives on, 50 ms bound)
+    records a timeout; the host reports KVC_ERR_DEVICE_TIMEOUT and the context
+    keeps working."""
+    ctx = small()
+    k, v, _ = kv(2, 40)
+    ctx.append([0, 1], k, v)
+    with pytest.raises(KvcError) as e:
+        ctx.check_wait_timeout(50)
+    assert e.value.status == kvc.KVC_ERR_DEVICE_TIMEOUT
+    ctx.sync()  # the status word was cleared
+    ctx.compress("random", np.array([20, 20], np.int32), 1)
+    ctx.sync()
+    assert list(ctx.lengths()[0]) == [20, 20]
+    ctx.close()
