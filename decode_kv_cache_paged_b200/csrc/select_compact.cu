@@ -47,6 +47,12 @@ namespace {
 #ifndef KVC_SC_UNROLL_LARGE
 #define KVC_SC_UNROLL_LARGE 8
 #endif
+// Segments with at most this many candidates run with 256 threads per CTA
+// (two CTAs per SM, so one CTA's select phase overlaps the other's copy);
+// larger ones with 512.
+#ifndef KVC_SC_NT256_MAX_N
+#define KVC_SC_NT256_MAX_N 4096
+#endif
 #ifndef KVC_SC_UNROLL_HOLE
 #define KVC_SC_UNROLL_HOLE 2
 #endif
@@ -454,7 +460,7 @@ cudaError_t launch_select_compact(const SelectCompactParams &p, int mode, int n_
   (void)max_m;
   if (n_seg_req <= 0) return cudaSuccess;
   const int var = (p.flags & kScHoleFill) ? kHoleFill : (p.flags & kScTieByPos) ? kOrderedPosTie : kOrderedSlotTie;
-  if (max_n <= 4096) return launch_nt<256, KVC_SC_UNROLL_SMALL>(p, mode, var, n_seg_req, max_n, s);
+  if (max_n <= KVC_SC_NT256_MAX_N) return launch_nt<256, KVC_SC_UNROLL_SMALL>(p, mode, var, n_seg_req, max_n, s);
   return launch_nt<512, KVC_SC_UNROLL_LARGE>(p, mode, var, n_seg_req, max_n, s);
 }
 

@@ -132,6 +132,49 @@ def test_many_layers_single_split():
     print(_run(w))
 
 
+def test_serving_full_size_sampled():
+    """The benchmarked step: 128 requests x 36 layers x 8 KV heads, 32 query heads, 2048 rows after a
+    round; 24 sampled (layer, request) pairs, every query head, against the oracle."""
+    w = wl.random_serving()
+    w.num_q_heads = 32
+    ctx = make_context(w)
+    gen = wl.Generator(w, "cuda")
+    wl.fill(ctx, w, gen, with_queries=False)
+    ctx.compress("random", w.budget.astype(np.int32), w.philox_seed)
+    g = torch.Generator(device="cuda").manual_seed(7)
+    q = torch.randn((w.num_layers, w.num_requests, 32, w.head_dim), generator=g, device="cuda").to(ctx.dtype)
+    out, lse = ctx.decode_attention(q)
+    ctx.sync()
+    lengths, _ = ctx.lengths()
+    rng = np.random.default_rng(3)
+    sc = 1 / np.sqrt(w.head_dim)
+    G = 32 // w.num_kv_heads
+    worst = 0.0
+    for _ in range(24):
+        l, r = int(rng.integers(w.num_layers)), int(rng.integers(w.num_requests))
+        L = int(lengths[r])
+        _, k, v = dense_layer(ctx, l, [r], L, lengths, with_kv=True)
+        k64 = k[0].float().cpu().numpy().astype(np.float64)
+        v64 = v[0].float().cpu().numpy().astype(np.float64)
+        q64 = q[l, r].float().cpu().numpy().astype(np.float64)
+        o_o, o_lse = oracle.decode_attention_gqa(q64, k64, v64, sc)
+        got = out[l, r].cpu().numpy().astype(np.float64)
+        got_lse = lse[l, r].cpu().numpy().astype(np.float64)
+        for hq in range(32):
+            h = hq // G
+            s = sc * (k64[h] @ q64[hq])
+            A = np.max(sc * (np.abs(k64[h]) @ np.abs(q64[hq])))
+            ds = LAM * np.sqrt(w.head_dim + 6) * U * A + U * np.max(s.max() - s) + 3 * U
+            acc = LAM * np.sqrt(L + 64) * U
+            tol = np.max(np.abs(v64[h]), axis=0) * (2 * ds + 2 * acc)
+            err = np.abs(got[hq] - o_o[hq])
+            assert np.all(err <= tol), (l, r, hq, float(err.max()))
+            assert abs(got_lse[hq] - o_lse[hq]) <= ds + acc + 4 * U * abs(o_lse[hq]), (l, r, hq)
+            worst = max(worst, float((err / tol).max()))
+    print("worst error / bound:", worst)
+    ctx.close()
+
+
 def test_every_row_counted_exactly():
     """Zero query, integer values: out = exact mean of the rows (one rounding)."""
     w = _workload()
