@@ -110,12 +110,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = smem_align<1024>(smem_raw);
   constexpr uint32_t kCBytes = CROWS * 256;          // beacon tile: CROWS rows x 128 bf16
   constexpr uint32_t kTileBytes = kTileKeys * 256;   // 32 KB
+  // TMEM accumulator buffers: 4 of 128 columns when a tile's products fit in
+  // 128 columns (at most 128 beacons), else 2 of 256; the epilogue group g
+  // drains the buffers b with b % 2 == g
+  constexpr int NACC = CROWS <= 128 ? 4 : 2;
+  constexpr uint32_t ACOLS = kTmemCols / NACC;
   uint8_t *cbuf = smem;                              // [NCB][2 K-halves][CROWS][128 B]
   uint8_t *kbuf = smem + NCB * kCBytes;              // [kStages][2][128][128 B]
   uint64_t *bars = reinterpret_cast<uint64_t *>(kbuf + kStages * kTileBytes);
   uint64_t *full = bars, *empty = bars + kStages;
-  uint64_t *acc_full = bars + 2 * kStages, *acc_empty = acc_full + 2;
-  uint64_t *c_full = acc_empty + 2, *c_empty = c_full + 2, *mma_done = c_empty + 2;
+  uint64_t *acc_full = bars + 2 * kStages, *acc_empty = acc_full + NACC;
+  uint64_t *c_full = acc_empty + NACC, *c_empty = c_full + 2, *mma_done = c_empty + 2;
   uint64_t *epi_bar = mma_done + 1;  // the 4 epilogue warps, once per segment
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(epi_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -129,9 +134,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NACC; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&c_full[i], 1);
       mbar_init(&c_empty[i], 1);
     }
@@ -238,13 +245,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         const uint32_t c_addr = smem_u32(cbuf + cb * kCBytes);
         for (int t = 0; t < g.n1 + g.n2; ++t, ++it, ++acc_it) {
-          const int st = it % kStages, buf = acc_it & 1;
+          const int st = it % kStages, buf = acc_it % NACC;
           ok = mbar_wait(&full[st], (it / kStages) & 1, abort_flag, p.status) &&
-               mbar_wait(&acc_empty[buf], ((acc_it >> 1) & 1) ^ 1, abort_flag, p.status);
+               mbar_wait(&acc_empty[buf], ((acc_it / NACC) & 1) ^ 1, abort_flag, p.status);
           if (!ok) break;
           tmem_fence_after();
           const uint32_t k_addr = smem_u32(kbuf + st * kTileBytes);
-          const uint32_t d = tmem_base + buf * 256;
+          const uint32_t d = tmem_base + buf * ACOLS;
           if (t < g.n1) {
             for (int half = 0; half * 128 < B; ++half)
               for (int kb = 0; kb < 2; ++kb)
@@ -294,9 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // pass 1: per-beacon online log2-sum-exp2 over this group's tiles
       float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
       for (int t = 0; t < g.n1; ++t, ++acc_it) {
-        const int buf = acc_it & 1;
-        if (buf != grp) continue;
-        ok = warp_wait(&acc_full[buf], (acc_it >> 1) & 1, abort_flag, p.status);
+        const int buf = acc_it % NACC;
+        if ((buf & 1) != grp) continue;
+        ok = warp_wait(&acc_full[buf], (acc_it / NACC) & 1, abort_flag, p.status);
         if (!ok) break;
         tmem_fence_after();
         const int nvalid = min(kTileKeys, g.L - t * kTileKeys);
@@ -307,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float &sum = half ? s1 : s0;
           for (int c0 = col_lo; c0 < col_lo + ncols; c0 += 64) {
             float v[64];
-            tmem_ld64(tmem_base + lane_addr + buf * 256 + half * 128 + c0, v);
+            tmem_ld64(tmem_base + lane_addr + buf * ACOLS + half * 128 + c0, v);
             const int nv = min(64, nvalid - c0);
             if (!mine || nv <= 0) continue;
             float mx[8];
@@ -376,9 +383,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // pass 2: per-key max over beacons of u - lse2 (this group's tiles)
       for (int t = 0; t < g.n2; ++t, ++acc_it) {
-        const int buf = acc_it & 1;
-        if (buf != grp) continue;
-        ok = warp_wait(&acc_full[buf], (acc_it >> 1) & 1, abort_flag, p.status);
+        const int buf = acc_it % NACC;
+        if ((buf & 1) != grp) continue;
+        ok = warp_wait(&acc_full[buf], (acc_it / NACC) & 1, abort_flag, p.status);
         if (!ok) break;
         tmem_fence_after();
         float bm[8];
@@ -387,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 8; ++i) bm[i] = trig ? 0.f : -INFINITY;
         for (int c0 = 0; c0 < B; c0 += 64) {
           float v[64];
-          tmem_ld64(tmem_base + lane_addr + buf * 256 + c0, v);
+          tmem_ld64(tmem_base + lane_addr + buf * ACOLS + c0, v);
           const float4 *l4 = reinterpret_cast<const float4 *>(lse_buf + c0);
           if (trig) {
             // cluster trigger: sum over beacons of share_b * 2^(u_bj - lse2_b)

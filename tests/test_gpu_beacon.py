@@ -211,6 +211,16 @@ def test_score_kernels_small(impl):
     print(impl, out)
 
 
+@pytest.mark.parametrize("B", [128, 192])
+def test_tcgen05_non_duplicated_beacon_tiles(B):
+    """128 beacons (one beacon copy per tile, four 128-column accumulator buffers) and 192 (two 128-row
+    halves, two 256-column buffers)."""
+    w = wl.beacon_serving(R=2, layers=2)
+    w.num_beacons = B
+    out = run_beacon(w, score_impl=2)
+    print(B, out)
+
+
 def test_tcgen05_256_beacons():
     """The 256-beacon path of the tensor-core kernel (two M=128 halves in pass 1)."""
     w = wl.scaled(wl.long_trace(), num_requests=1, num_layers=2)
