@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
   constexpr int D = 128;
   const int B = p.B, NP = p.W * p.G;
   const int nh = (B + 127) / 128;        // halves of 128 beacons
+  const bool dup = B <= 64;              // one-hot rows written twice (see below)
   const uint32_t acol = B <= 128 ? 128u : 256u;  // sums of half h at columns acol + 128 h
   uint8_t *xs = smem;                    // [2 K-blocks][128 points][128 B]
   uint8_t *chi = xs + 32768;             // [2][B][128 B]
@@ -117,8 +118,14 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
   // 32 beacons' loads in flight at once
   for (int b0 = 0; b0 < B; b0 += 32) {  // B is a multiple of 32
     float c[32];
+    if (ud.init) {
 #pragma unroll
-    for (int u = 0; u < 32; ++u) c[u] = c_old(b0 + u, tid);
+      for (int u = 0; u < 32; ++u) c[u] = c_old(b0 + u, tid);
+    } else {
+      // no branch between the loads, so all 32 are in flight together
+#pragma unroll
+      for (int u = 0; u < 32; ++u) c[u] = gbeac[(b0 + u) * D + tid];
+    }
     const int kb = tid >> 6, k = tid & 63;
 #pragma unroll
     for (int u8 = 0; u8 < 32; u8 += 8) {
@@ -199,11 +206,18 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
       if (p.assign_out) p.assign_out[seg * (int64_t)NP + pt] = besti;
       atomicAdd(&cnt[besti], 1);
     }
-    // this point's entry of the one-hot tile (row = beacon within its half)
+    // this point's entry of the one-hot tile (row = beacon within its half);
+    // with at most 64 beacons every row is written twice (rows b and b + 64),
+    // so the sums of beacon b sit in TMEM lanes b and b + 64 and all four
+    // warps take part in the running mean
     const uint32_t oh_off = (uint32_t)(tid >> 6) * 16384u + sw128_off(besti & 127, tid & 63);
+    const uint32_t oh_dup = dup ? (uint32_t)(tid >> 6) * 16384u + sw128_off(besti + 64, tid & 63) : oh_off;
     for (int hh = 0; hh < nh; ++hh) {
       const bool here = valid && (besti >> 7) == hh;
-      if (here) *reinterpret_cast<__nv_bfloat16 *>(asum + oh_off) = __float2bfloat16_rn(1.f);
+      if (here) {
+        *reinterpret_cast<__nv_bfloat16 *>(asum + oh_off) = __float2bfloat16_rn(1.f);
+        *reinterpret_cast<__nv_bfloat16 *>(asum + oh_dup) = __float2bfloat16_rn(1.f);
+      }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tmem_fence_before();
       __syncthreads();
@@ -223,7 +237,10 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
       ++phase;
       __syncthreads();  // the product has read the one-hot tile
       if (*abort_flag) break;
-      if (here) *reinterpret_cast<__nv_bfloat16 *>(asum + oh_off) = __float2bfloat16_rn(0.f);
+      if (here) {
+        *reinterpret_cast<__nv_bfloat16 *>(asum + oh_off) = __float2bfloat16_rn(0.f);
+        *reinterpret_cast<__nv_bfloat16 *>(asum + oh_dup) = __float2bfloat16_rn(0.f);
+      }
     }
     if (*abort_flag) break;
     tmem_fence_before();
@@ -237,10 +254,14 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
     // values loaded together
     tmem_fence_after();
     for (int hh = 0; hh < nh; ++hh) {
-      const int b = 128 * hh + tid;
+      // thread t: beacon 128 hh + t, all dimensions; or, with the duplicated
+      // rows, beacon t % 64 and the dimension half t / 64
+      const int b = dup ? (tid & 63) : 128 * hh + tid;
+      const int dlo = dup ? (tid >> 6) * (D / 2) : 0, dhi = dup ? dlo + D / 2 : D;
       const bool mine = b < B;
       const int m = mine ? cnt[b] : 0;
       const int n = (mine && !ud.init) ? gcnt[b] : 0;
+      __syncthreads();  // every thread has read the old count before any is rewritten
       float4 *g4 = reinterpret_cast<float4 *>(gbeac + (int64_t)b * D);
       __nv_bfloat162 *s2 = reinterpret_cast<__nv_bfloat162 *>(reinterpret_cast<__nv_bfloat16 *>(p.beacons_s) +
                                                                (seg * B + b) * D);
@@ -252,9 +273,9 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
 #pragma unroll
           for (int q = 0; q < 8; ++q) ov[q] = g4[c0 / 4 + q];
       };
-      load_old(0);
+      load_old(dlo);
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = dlo; c0 < dhi; c0 += 32) {
         float sm[32];
         tmem_ld32(tmem_base + lane_addr + acol + 128u * hh + c0, sm);  // warp-collective
         float v[32];
@@ -269,7 +290,7 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
             }
           }
         }
-        if (c0 + 32 < D) load_old(c0 + 32);
+        if (c0 + 32 < dhi) load_old(c0 + 32);
         if (mine) {
           if (m > 0)
 #pragma unroll
@@ -282,7 +303,7 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
           }
         }
       }
-      if (mine) {
+      if (mine && dlo == 0) {
         gcnt[b] = n + m;
         p.trig[seg * B + b] = (float)m / (float)n_pts;
       }
