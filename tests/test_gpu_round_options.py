@@ -46,10 +46,10 @@ def _pre_slot_of(pre_pos_seg: np.ndarray, post_pos_seg: np.ndarray) -> np.ndarra
     return idx
 
 
-def run_option_rounds(w, selector, plan, seed, kv_layers=(0,), check_scores_n=300):
+def run_option_rounds(w, selector, plan, seed, kv_layers=(0,), check_scores_n=300, extra_pages=0):
     """plan: list of per-round dicts with keys sinks (None or S), block, compaction."""
     headroom = max(0, int(max(w.budget.max(), w.prompt.max()) + w.trigger - w.length.max()))
-    ctx = make_context(w, headroom=headroom)
+    ctx = make_context(w, headroom=headroom, extra_pages=extra_pages)
     gen = wl.Generator(w, "cuda")
     wl.fill(ctx, w, gen, with_queries=False)
     R, Ly, H = w.num_requests, w.num_layers, w.num_kv_heads
