@@ -21,11 +21,16 @@
 //     warp's 2-slot ring, completing on a transaction-count mbarrier.  Warps
 //     keep their own running max and sums, so no block-wide barrier is taken
 //     until the four warps' states are merged at the end.
-//   * Scores: two lanes per row, each half the dimensions; the 8 lanes of a
-//     quarter-warp take 8 rows and rotate their chunk order by the row, so
-//     their reads of K (256-byte rows) and of the query (48-byte chunk
-//     stride) each fall in 8 different bank groups.  Online softmax in base
-//     2 with the scale folded into q.
+//   * Scores: every lane owns one 16-byte chunk of the row (the same chunk
+//     for every row it scores) and keeps that chunk of the G query rows in
+//     registers, so the only shared-memory reads of the score step are the
+//     K rows themselves, a quarter-warp reading 128 consecutive bytes.  The
+//     lanes of a row then sum their partial dot products with a butterfly
+//     reduce-scatter (each exchange halves the sums a lane holds), ending
+//     with each lane holding whole scores of one row for a few heads.  The
+//     query used to be re-read from shared memory for every chunk, which
+//     made the shared-memory data pipe the limit.  Online softmax in base 2
+//     with the scale folded into q.
 //   * P.V: each lane owns 8-byte segments of a row for all G heads.
 //   * Products and sums use the packed two-wide fp32 FMA of sm_100 (the
 //     same rounding as two scalar FMAs, half the instructions).
@@ -89,10 +94,8 @@ template <typename T, int D, int G>
 struct AttnShape {
   static constexpr int kRowBytes = D * (int)sizeof(T);
   static constexpr int kChunks = kRowBytes / 16;           // 16-byte chunks per row
-  static constexpr int kHalfChunks = kChunks / 2;          // per scoring lane
   static constexpr int kPairs = 16 / (int)sizeof(T) / 2;   // element pairs per chunk
   static constexpr int kEpc = 2 * kPairs;                  // elements per chunk
-  static constexpr int kQStride = 12;                      // floats per query chunk in shared memory
   static constexpr int kPageBytes = kPage * kRowBytes;     // one page of K (or V): 16 rows, contiguous
   static constexpr int kSlotBytes = 2 * kPageBytes;        // K and V of one page
   static constexpr int kWarpStages = KVC_ATTN_STAGES;      // page slots per warp
@@ -104,11 +107,51 @@ struct AttnShape {
   static constexpr int kRowPar = kRowBytes >= 256 ? 1 : 256 / kRowBytes;
   static constexpr int kVp = 8 / (int)sizeof(T) / 2;       // element pairs per 8-byte segment
   static constexpr int kAccPairs = kSeg * kVp;             // accumulator pairs per head per lane
+  // scores: kLpr lanes per row, one chunk each; a warp scores kRowGroups rows
+  // at once; a lane's partial sums are reduced kRb rows (kNv sums) at a time
+  static constexpr int kLpr = kChunks;
+  static constexpr int kRowGroups = 32 / kLpr;
+  static constexpr int kRowsPerGroup = kPage / kRowGroups;
+  static constexpr int kRb = kRowsPerGroup < 32 / G ? kRowsPerGroup : 32 / G;
+  static constexpr int kBatches = kRowsPerGroup / kRb;
+  static constexpr int kNv = kRb * G;
+  // after the reduce-scatter a lane holds kKeep whole scores (consecutive
+  // heads of one row); kDup lanes hold each score when kNv < kLpr
+  static constexpr int kKeep = kNv >= kLpr ? kNv / kLpr : 1;
+  static constexpr int kDup = kNv >= kLpr ? 1 : kLpr / kNv;
+  // lanes xor-apart by at least kHeadMask hold the same heads (other rows)
+  static constexpr int kHeadMask = kLpr / kRb;
   static_assert(kRowBytes >= 128 && kRowBytes <= 512, "row size");
-  static_assert((kHalfChunks & (kHalfChunks - 1)) == 0, "chunk rotation needs a power of two");
+  static_assert(kKeep < G || G == 1, "a lane keeps part of the heads of one row");
+  static_assert(kHeadMask >= 2 && kHeadMask <= 32 && kDup <= kHeadMask, "lane classes");
   static_assert((size_t)kWarps * G * D * 4 <= (size_t)kWarps * kWarpStages * kSlotBytes,
                 "the merge buffer reuses the page slots");
 };
+
+// Reduce-scatter of N partial sums over the lanes xor M, M/2, ..., 1 apart:
+// each exchange sends half of the sums still held to the partner and adds
+// the partner's half of its own; once a lane holds one sum the remaining
+// exchanges add the partner's copy of it.  Afterwards, with M = the lanes of
+// a row / 2, lane c of the row holds the whole sums of entries
+// c * N / (2M) + k, k < max(1, N / (2M)), in v[k].
+template <int N, int M, int NV>
+__device__ __forceinline__ void reduce_scatter(float (&v)[NV], int lane) {
+  if constexpr (M >= 1) {
+    if constexpr (N > 1) {
+      const bool upper = (lane & M) != 0;
+#pragma unroll
+      for (int k = 0; k < N / 2; ++k) {
+        const float send = upper ? v[k] : v[k + N / 2];
+        const float keep = upper ? v[k + N / 2] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, M);
+      }
+      reduce_scatter<N / 2, M / 2>(v, lane);
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], M);
+      reduce_scatter<1, M / 2>(v, lane);
+    }
+  }
+}
 
 // Each of the 4 warps walks every 4th page of the CTA's split through its own
 // 2-slot ring (K and V of one page per slot), with its own running max and
@@ -116,13 +159,11 @@ struct AttnShape {
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads) decode_attention_kernel(DecodeAttnParams p) {
   using S = AttnShape<T, D, G>;
-  constexpr int W = S::kWarps, NS = S::kWarpStages;
+  constexpr int W = S::kWarps, NS = S::kWarpStages, KEEP = S::kKeep;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_align<128>(smem_raw);
-  // query chunk c of head g at q_s[g][c]: 48-byte chunk stride, so the 8
-  // lanes of a quarter-warp reading 8 different chunks hit 8 bank groups
-  __shared__ __align__(16) float q_s[G][S::kChunks][S::kQStride];
-  __shared__ __align__(16) float p_s[W][kPage][G];
+  __shared__ __align__(16) float p_s[W][kPage][G];  // the page's softmax weights
+  __shared__ __align__(16) float a_s[W][G];         // the page's rescale factors
   __shared__ float m_s[W][G], l_s[W][G];
   __shared__ __align__(8) uint64_t full[W][NS];
   __shared__ int abort_flag_s;
@@ -149,13 +190,6 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(DecodeAttnPa
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  {  // this CTA's G query rows, pre-scaled into base 2
-    const T *q = reinterpret_cast<const T *>(p.q) + (((int64_t)lc * p.R + r) * p.hq + (int64_t)h * G) * D;
-    for (int i = tid; i < G * D; i += kThreads) {
-      const int g = i / D, e = i % D;
-      q_s[g][e / S::kEpc][e % S::kEpc] = to_float(q[i]) * p.qscale;
-    }
-  }
   __syncthreads();
 
   // lanes 0 and 1 copy page k's K and V rows (each one contiguous block of
@@ -174,18 +208,37 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(DecodeAttnPa
   };
   for (int k = 0; k < min(n_my, NS); ++k) issue_page(k);
 
-  float m_run[G], l_lane[G];
+  // scoring lanes: chunk c of the rows of row group grp; the whole scores a
+  // lane ends with are of entries e0 + k (row e0 / G of a batch, heads g0 + k)
+  const int c = lane % S::kLpr;
+  const int grp = lane / S::kLpr;
+  const int e0 = (c / S::kDup) * KEEP;
+  const int g0 = e0 % G;
+  const bool writer = (c % S::kDup) == 0;  // one lane of each set of copies stores
+
+  // chunk c of this KV head's G query rows, scaled into base 2, in registers
+  float2 qr[G][S::kPairs];
+  {
+    const T *q = reinterpret_cast<const T *>(p.q) + (((int64_t)lc * p.R + r) * p.hq + (int64_t)h * G) * D;
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < S::kPairs; ++e)
+        qr[g][e] = make_float2(to_float(q[g * D + c * S::kEpc + 2 * e]) * p.qscale,
+                               to_float(q[g * D + c * S::kEpc + 2 * e + 1]) * p.qscale);
+  }
+
+  float m_run[KEEP], l_lane[KEEP];
   float2 acc[G][S::kAccPairs];
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m_run[g] = -INFINITY;
-    l_lane[g] = 0.f;
+  for (int k = 0; k < KEEP; ++k) {
+    m_run[k] = -INFINITY;
+    l_lane[k] = 0.f;
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int e = 0; e < S::kAccPairs; ++e) acc[g][e] = make_float2(0.f, 0.f);
-  }
-  // scoring: lanes l and l^8 share row rr, each takes half of its chunks
-  const int half = (lane >> 3) & 1;
-  const int rr = (lane & 7) + 8 * (lane >> 4);
   // P.V: row group and 8-byte segment of this lane
   const int vgrp = lane / (32 / S::kRowPar);
   const int vlane = lane % (32 / S::kRowPar);
@@ -199,67 +252,74 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(DecodeAttnPa
     const uint8_t *vp = kp + S::kPageBytes;
     const int valid = min(kPage, len - (pg0 + warp + k * W) * kPage);
 
-    // 1. scores of row rr
-    float2 s2[G];
+    // 1. scores: partial dot products of chunk c, reduced across the row's lanes
+    float sv[S::kBatches][KEEP];
 #pragma unroll
-    for (int g = 0; g < G; ++g) s2[g] = make_float2(0.f, 0.f);
+    for (int b = 0; b < S::kBatches; ++b) {
+      float part[S::kNv];  // entry i * G + g: row i of the batch, head g
 #pragma unroll
-    for (int i = 0; i < S::kHalfChunks; ++i) {
-      // lanes of a quarter-warp take 8 rows and rotate the chunk order by the
-      // row, so their 16-byte reads fall in 8 different bank groups
-      const int c = half * S::kHalfChunks + ((i + rr) & (S::kHalfChunks - 1));
-      float2 x[S::kPairs];
-      load_chunk2<T>(kp + rr * S::kRowBytes + c * 16, x);
+      for (int i = 0; i < S::kRb; ++i) {
+        const int row = grp * S::kRowsPerGroup + b * S::kRb + i;
+        float2 x[S::kPairs];
+        load_chunk2<T>(kp + row * S::kRowBytes + c * 16, x);
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
+        for (int g = 0; g < G; ++g) {
+          float2 t = __fmul2_rn(qr[g][0], x[0]);
 #pragma unroll
-        for (int e = 0; e < S::kPairs; e += 2) {
-          const float4 qv = *reinterpret_cast<const float4 *>(&q_s[g][c][2 * e]);
-          s2[g] = __ffma2_rn(make_float2(qv.x, qv.y), x[e], s2[g]);
-          s2[g] = __ffma2_rn(make_float2(qv.z, qv.w), x[e + 1], s2[g]);
+          for (int e = 1; e < S::kPairs; ++e) t = __ffma2_rn(qr[g][e], x[e], t);
+          part[i * G + g] = t.x + t.y;
         }
       }
+      reduce_scatter<S::kNv, S::kLpr / 2>(part, lane);
+      const int row = grp * S::kRowsPerGroup + b * S::kRb + e0 / G;
+#pragma unroll
+      for (int kk = 0; kk < KEEP; ++kk) sv[b][kk] = row < valid ? part[kk] : -INFINITY;
     }
-    const bool ok = rr < valid;
-    float pw[G], alpha[G];
+
+    // 2. online softmax per head: the max over the lanes holding that head
+    float alpha[KEEP];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float sg = s2[g].x + s2[g].y;
-      sg += __shfl_xor_sync(0xffffffffu, sg, 8);
-      sg = ok ? sg : -INFINITY;
-      float mx = sg;
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      const float m_new = fmaxf(m_run[g], mx);  // finite: a page has a valid row
-      alpha[g] = exp2f(m_run[g] - m_new);
-      m_run[g] = m_new;
-      pw[g] = ok ? exp2f(sg - m_new) : 0.f;
-      l_lane[g] = fmaf(l_lane[g], alpha[g], half == 0 ? pw[g] : 0.f);
-    }
-    if (half == 0) {
-      if constexpr (G % 4 == 0) {
+    for (int kk = 0; kk < KEEP; ++kk) {
+      float mx = sv[0][kk];
 #pragma unroll
-        for (int g = 0; g < G; g += 4)
-          *reinterpret_cast<float4 *>(&p_s[warp][rr][g]) = make_float4(pw[g], pw[g + 1], pw[g + 2], pw[g + 3]);
-      } else {
+      for (int b = 1; b < S::kBatches; ++b) mx = fmaxf(mx, sv[b][kk]);
 #pragma unroll
-        for (int g = 0; g < G; ++g) p_s[warp][rr][g] = pw[g];
+      for (int m = S::kHeadMask; m < 32; m <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+      const float m_new = fmaxf(m_run[kk], mx);  // finite: a page has a valid row
+      alpha[kk] = exp2f(m_run[kk] - m_new);
+      m_run[kk] = m_new;
+      float ps = 0.f;
+#pragma unroll
+      for (int b = 0; b < S::kBatches; ++b) {
+        sv[b][kk] = exp2f(sv[b][kk] - m_new);  // 0 for rows past the end
+        ps += sv[b][kk];
       }
+      l_lane[kk] = fmaf(l_lane[kk], alpha[kk], ps);
+    }
+    if (writer) {
+#pragma unroll
+      for (int b = 0; b < S::kBatches; ++b) {
+        float *dst = &p_s[warp][grp * S::kRowsPerGroup + b * S::kRb + e0 / G][g0];
+        if constexpr (KEEP == 4)
+          *reinterpret_cast<float4 *>(dst) = make_float4(sv[b][0], sv[b][1], sv[b][2], sv[b][3]);
+        else if constexpr (KEEP == 2)
+          *reinterpret_cast<float2 *>(dst) = make_float2(sv[b][0], sv[b][1]);
+        else
+#pragma unroll
+          for (int kk = 0; kk < KEEP; ++kk) dst[kk] = sv[b][kk];
+      }
+      if (lane < S::kHeadMask)  // lanes below kHeadMask hold every head once
+#pragma unroll
+        for (int kk = 0; kk < KEEP; ++kk) a_s[warp][g0 + kk] = alpha[kk];
     }
     __syncwarp();
-    // 2. acc = acc * alpha + P.V over the page's valid rows
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int e = 0; e < S::kAccPairs; ++e) acc[g][e] = __fmul2_rn(acc[g][e], make_float2(alpha[g], alpha[g]));
-    auto pv_row = [&](int vr) {
-      float w[G];
+
+    // 3. acc = acc * alpha + P.V over the page's valid rows
+    auto read_g = [&](const float *src, float (&w)[G]) {
       if constexpr (G % 4 == 0) {
 #pragma unroll
         for (int g = 0; g < G; g += 4) {
-          const float4 w4 = *reinterpret_cast<const float4 *>(&p_s[warp][vr][g]);
+          const float4 w4 = *reinterpret_cast<const float4 *>(src + g);
           w[g] = w4.x;
           w[g + 1] = w4.y;
           w[g + 2] = w4.z;
@@ -267,8 +327,20 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(DecodeAttnPa
         }
       } else {
 #pragma unroll
-        for (int g = 0; g < G; ++g) w[g] = p_s[warp][vr][g];
+        for (int g = 0; g < G; ++g) w[g] = src[g];
       }
+    };
+    {
+      float a[G];
+      read_g(a_s[warp], a);
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < S::kAccPairs; ++e) acc[g][e] = __fmul2_rn(acc[g][e], make_float2(a[g], a[g]));
+    }
+    auto pv_row = [&](int vr) {
+      float w[G];
+      read_g(p_s[warp][vr], w);
 #pragma unroll
       for (int sg = 0; sg < S::kSeg; ++sg) {
         const int byte = sg * 256 + vlane * 8;  // 8-byte segment within the row
@@ -282,14 +354,14 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(DecodeAttnPa
       }
     };
     if (valid == kPage) {
-      // full page (all but a segment's last): rows and swizzle offsets known at compile time
+      // full page (all but a segment's last): rows known at compile time
 #pragma unroll
       for (int i = 0; i < kPage / S::kRowPar; ++i) pv_row(i * S::kRowPar + vgrp);
     } else {
 #pragma unroll 1
       for (int vr = vgrp; vr < valid; vr += S::kRowPar) pv_row(vr);
     }
-    __syncwarp();  // the slot and p_s are free again
+    __syncwarp();  // the slot, p_s and a_s are free again
     if (k + NS < n_my) issue_page(k + NS);
   }
   if (k < n_my) {
@@ -300,15 +372,15 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(DecodeAttnPa
         mbar_wait(&full[warp][j % NS], (uint32_t)((j / NS) & 1), abort_flag, p.status, false);
   }
 
-  // 3. merge the warps: each writes (max, sum, accumulators)
+  // 4. merge the warps: each writes (max, sum, accumulators)
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float ls = l_lane[g];
+  for (int kk = 0; kk < KEEP; ++kk) {
+    float ls = l_lane[kk];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-    if (lane == 0) {
-      m_s[warp][g] = m_run[g];
-      l_s[warp][g] = ls;
+    for (int m = S::kHeadMask; m < 32; m <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, m);
+    if (writer && lane < S::kHeadMask) {
+      m_s[warp][g0 + kk] = m_run[kk];
+      l_s[warp][g0 + kk] = ls;
     }
   }
   if constexpr (S::kRowPar > 1) {
