@@ -27,11 +27,15 @@
 // the tensor map covers the whole pool as rows of 128 bf16, 128-byte
 // swizzle); warp 1 issues the MMAs (one elected lane) and commits them to
 // mbarriers; warps 2-9 run the epilogue in two groups of four, group g taking
-// the tiles whose accumulator is in TMEM buffer g (tcgen05.ld of 64 columns
-// at a time; sums and maxima in 8 independent partials; the per-beacon
-// partial (max, sum) of the groups merged once per segment).
-// Key tiles rotate through 4 shared-memory stages; the accumulators through
-// two 256-column TMEM buffers.  No load uses cluster multicast.
+// the tiles whose accumulator is in TMEM buffers of parity g (tcgen05.ld of
+// 64 columns at a time; sums and maxima in 8 independent partials; the
+// per-beacon partial (max, sum) of the groups merged once per segment).
+// Pass 1 adds a full 64-column chunk as sum 2^(u - m) against the running
+// reference m with no max pass first; only a chunk whose sum would pass
+// 2^64 (a new maximum far above m) or a partial chunk takes the max-then-
+// rescale step.  Key tiles rotate through 4 shared-memory stages; the
+// accumulators through four 128-column TMEM buffers (at most 128 beacons)
+// or two of 256.  No load uses cluster multicast.
 // Every mbarrier wait is bounded (2 s of %globaltimer): on expiry the kernel
 // records KVC_ERR_DEVICE_TIMEOUT in the status word, the other roles see the
 // abort flag and leave, and TMEM is released before the CTA exits.
@@ -307,7 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tmem_fence_after();
         const int nvalid = min(kTileKeys, g.L - t * kTileKeys);
-        for (int half = 0; half * 128 < B; ++half) {
+        const int nhalf = (B + 127) / 128;
+        for (int half = 0; half < nhalf; ++half) {
           const int b = half * 128 + (dup ? (row & 63) : row);
           const bool mine = b < B;
           float &m = half ? m1 : m0;
@@ -315,8 +320,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c0 = col_lo; c0 < col_lo + ncols; c0 += 64) {
             float v[64];
             tmem_ld64(tmem_base + lane_addr + buf * ACOLS + half * 128 + c0, v);
+            if (half == nhalf - 1 && c0 + 64 >= col_lo + ncols) {
+              // the tile's last load has landed in registers: hand the
+              // buffer back to the MMA warp before the arithmetic
+              tmem_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            }
             const int nv = min(64, nvalid - c0);
             if (!mine || nv <= 0) continue;
+            if (nv == 64 && m != -INFINITY) {
+              // full chunk against the running reference m, with no max
+              // pass: sum stays sum_j 2^(u_j - m) whether or not u_j <= m,
+              // and a chunk sum within 2^64 cannot lose the total to
+              // overflow; a larger one (a new maximum far above m, or a
+              // NaN) takes the exact path below
+              // (two-wide packed FMA and add: the rounding of two scalar ops)
+              float2 ps[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) ps[i] = make_float2(0.f, 0.f);
+              const float2 a2 = make_float2(alpha, alpha), nm2 = make_float2(-m, -m);
+#pragma unroll
+              for (int i = 0; i < 64; i += 2) {
+                const float2 t = __ffma2_rn(make_float2(v[i], v[i + 1]), a2, nm2);
+                ps[(i >> 1) & 3] = __fadd2_rn(ps[(i >> 1) & 3], make_float2(exp2f(t.x), exp2f(t.y)));
+              }
+              const float cs = ((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) + ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y));
+              if (cs <= 0x1p64f) {
+                sum += cs;
+                continue;
+              }
+            }
             float mx[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
@@ -338,9 +372,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
           }
         }
-        tmem_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
       }
       if (!ok) break;
       // merge the partial (max, sum) of each beacon over groups and copies
@@ -368,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (pm != -INFINITY) ss += part[(k * 2 + 1) * 256 + b] * exp2f(pm - mm);
             }
             const float l2 = mm + log2f(ss);
-            lse_buf[b] = l2;
+            lse_buf[b] = -l2;  // negated: pass 2 adds it in one packed FMA
             if (p.trig) w_buf[b] = p.trig[g.seg_flat * B + b];
             if (p.lse_out) p.lse_out[g.seg_flat * B + b] = l2 * 0.69314718055994531f;
             if (l2 != l2) atomicCAS(p.status, kDevOk, kDevNaN);
@@ -390,11 +421,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_fence_after();
         float bm[8];
         const bool trig = p.trig != nullptr;
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
         for (int i = 0; i < 8; ++i) bm[i] = trig ? 0.f : -INFINITY;
         for (int c0 = 0; c0 < B; c0 += 64) {
           float v[64];
           tmem_ld64(tmem_base + lane_addr + buf * ACOLS + c0, v);
+          if (c0 + 64 >= B) {  // the tile's last load: hand the buffer back
+            tmem_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          }
           const float4 *l4 = reinterpret_cast<const float4 *>(lse_buf + c0);
           if (trig) {
             // cluster trigger: sum over beacons of share_b * 2^(u_bj - lse2_b)
@@ -402,25 +439,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i4 = 0; i4 < 16; ++i4) {
               const float4 L4 = l4[i4], W4 = w4[i4];
-              bm[(4 * i4) & 7] = fmaf(W4.x, exp2f(fmaf(v[4 * i4], alpha, -L4.x)), bm[(4 * i4) & 7]);
-              bm[(4 * i4 + 1) & 7] = fmaf(W4.y, exp2f(fmaf(v[4 * i4 + 1], alpha, -L4.y)), bm[(4 * i4 + 1) & 7]);
-              bm[(4 * i4 + 2) & 7] = fmaf(W4.z, exp2f(fmaf(v[4 * i4 + 2], alpha, -L4.z)), bm[(4 * i4 + 2) & 7]);
-              bm[(4 * i4 + 3) & 7] = fmaf(W4.w, exp2f(fmaf(v[4 * i4 + 3], alpha, -L4.w)), bm[(4 * i4 + 3) & 7]);
+              const float2 t01 = __ffma2_rn(make_float2(v[4 * i4], v[4 * i4 + 1]), a2, make_float2(L4.x, L4.y));
+              const float2 t23 = __ffma2_rn(make_float2(v[4 * i4 + 2], v[4 * i4 + 3]), a2, make_float2(L4.z, L4.w));
+              bm[(4 * i4) & 7] = fmaf(W4.x, exp2f(t01.x), bm[(4 * i4) & 7]);
+              bm[(4 * i4 + 1) & 7] = fmaf(W4.y, exp2f(t01.y), bm[(4 * i4 + 1) & 7]);
+              bm[(4 * i4 + 2) & 7] = fmaf(W4.z, exp2f(t23.x), bm[(4 * i4 + 2) & 7]);
+              bm[(4 * i4 + 3) & 7] = fmaf(W4.w, exp2f(t23.y), bm[(4 * i4 + 3) & 7]);
             }
           } else {
 #pragma unroll
             for (int i4 = 0; i4 < 16; ++i4) {
               const float4 L4 = l4[i4];
-              bm[(4 * i4) & 7] = fmaxf(bm[(4 * i4) & 7], fmaf(v[4 * i4], alpha, -L4.x));
-              bm[(4 * i4 + 1) & 7] = fmaxf(bm[(4 * i4 + 1) & 7], fmaf(v[4 * i4 + 1], alpha, -L4.y));
-              bm[(4 * i4 + 2) & 7] = fmaxf(bm[(4 * i4 + 2) & 7], fmaf(v[4 * i4 + 2], alpha, -L4.z));
-              bm[(4 * i4 + 3) & 7] = fmaxf(bm[(4 * i4 + 3) & 7], fmaf(v[4 * i4 + 3], alpha, -L4.w));
+              const float2 t01 = __ffma2_rn(make_float2(v[4 * i4], v[4 * i4 + 1]), a2, make_float2(L4.x, L4.y));
+              const float2 t23 = __ffma2_rn(make_float2(v[4 * i4 + 2], v[4 * i4 + 3]), a2, make_float2(L4.z, L4.w));
+              bm[(4 * i4) & 7] = fmaxf(bm[(4 * i4) & 7], t01.x);
+              bm[(4 * i4 + 1) & 7] = fmaxf(bm[(4 * i4 + 1) & 7], t01.y);
+              bm[(4 * i4 + 2) & 7] = fmaxf(bm[(4 * i4 + 2) & 7], t23.x);
+              bm[(4 * i4 + 3) & 7] = fmaxf(bm[(4 * i4 + 3) & 7], t23.y);
             }
           }
         }
-        tmem_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
         const int j = g.tile_of(g.n1 + t) * kTileKeys + row;
         if (j >= g.P && j < g.L) {
           const float sc =

@@ -45,7 +45,7 @@ def _fill_recording(ctx, w, gen):
     return qwin
 
 
-def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered", selector="beacon"):
+def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered", selector="beacon", k_hook=None):
     ctx = make_context(w)
     if score_impl is not None:
         ctx.set_option(0, score_impl)
@@ -88,6 +88,8 @@ def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered"
         assert np.array_equal(g_trig[r, l, h], share), (r, l, h)
         assert np.allclose(g_beacons[r, l, h], c_s, rtol=1e-5, atol=1e-6), (r, l, h)
     # the round
+    if k_hook is not None:
+        k_hook(ctx)  # edits the cached keys before the pre-round snapshot
     lengths, prompts = ctx.lengths()
     cap = int(lengths.max())
     need_l = sorted({l for (_, l, _) in segs})
@@ -229,6 +231,38 @@ def test_tcgen05_256_beacons():
     w.prompt = np.array([77])
     out = run_beacon(w, score_impl=2)
     print(out)
+
+
+def _plant_dominant_keys(slots, z):
+    """Overwrites the keys at `slots` of every segment with a multiple of the segment's scoring beacon 0,
+    scaled so that z_0j = c_0.k_j / sqrt(d) is about z: a logit far above every earlier one."""
+    def hook(ctx):
+        st = ctx.state_tensors()
+        bt = st["block_table"].cpu().numpy()
+        c0 = st["beacons_scoring"][:, :, :, 0, :].float()  # [R, Ly, H, d]
+        R, Ly, H, d = c0.shape
+        for r in range(R):
+            for l in range(Ly):
+                for h in range(H):
+                    lam = z * d ** 0.5 / float((c0[r, l, h] ** 2).sum())
+                    for j in slots:
+                        ctx.k_pool[l, int(bt[r, j // 16]), h, j % 16] = (lam * c0[r, l, h]).to(ctx.dtype)
+        ctx.sync()
+    return hook
+
+
+@pytest.mark.parametrize("B", [64, 256])
+def test_tcgen05_logit_far_above_running_max(B):
+    """Keys whose logit sits ~200 above every earlier key of the segment: the pass-1 chunk sum against the
+    running reference would overflow, so that chunk must take the exact rescaling path.  Slot 1000 lies in
+    a full 64-key chunk of a full tile, slot 3100 in a later one."""
+    w = wl.scaled(wl.long_trace(), num_requests=1, num_layers=2)
+    w.num_beacons = B
+    w.length = np.array([4133])
+    w.budget = np.array([1000])
+    w.prompt = np.array([77])
+    out = run_beacon(w, score_impl=2, k_hook=_plant_dominant_keys([1000, 3100], 200.0))
+    print(B, out)
 
 
 @pytest.mark.parametrize("impl,B", [(1, 64), (2, 64), (2, 32), (2, 96), (2, 128), (2, 256)],
