@@ -158,6 +158,18 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
   // sums: A = one-hot^T (K-major), B operand = X (MN-major, transpose bit 16)
   const uint32_t idesc_sum = idesc_bf16_f32(128, D) | (1u << 16);
   const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+  // the running mean's first 64 old values and old count of this thread's
+  // first beacon (mapping as in the running mean below), loaded now so that
+  // they arrive while the point tiles run
+  const int b_first = dup ? (tid & 63) : tid;
+  float4 ov0[16];
+  int n_first = 0;
+  if (!ud.init && b_first < B) {
+    const float4 *src = reinterpret_cast<const float4 *>(gbeac + (int64_t)b_first * D + (dup ? (tid >> 6) * (D / 2) : 0));
+#pragma unroll
+    for (int q = 0; q < 16; ++q) ov0[q] = src[q];
+    n_first = gcnt[b_first];
+  }
   bool nan = false;
   int phase = 0;
   for (int p0 = 0; p0 < n_pts; p0 += 128) {
@@ -257,25 +269,29 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
       // thread t: beacon 128 hh + t, all dimensions; or, with the duplicated
       // rows, beacon t % 64 and the dimension half t / 64
       const int b = dup ? (tid & 63) : 128 * hh + tid;
-      const int dlo = dup ? (tid >> 6) * (D / 2) : 0, dhi = dup ? dlo + D / 2 : D;
+      const int dlo = dup ? (tid >> 6) * (D / 2) : 0;
+      const int nchunk = dup ? 2 : 4;  // 32-dimension chunks of this thread (CTA-uniform)
       const bool mine = b < B;
       const int m = mine ? cnt[b] : 0;
-      const int n = (mine && !ud.init) ? gcnt[b] : 0;
+      const int n = hh == 0 ? n_first : ((mine && !ud.init) ? gcnt[b] : 0);
       __syncthreads();  // every thread has read the old count before any is rewritten
       float4 *g4 = reinterpret_cast<float4 *>(gbeac + (int64_t)b * D);
       __nv_bfloat162 *s2 = reinterpret_cast<__nv_bfloat162 *>(reinterpret_cast<__nv_bfloat16 *>(p.beacons_s) +
                                                                (seg * B + b) * D);
-      // old values of 32 dimensions, the next chunk's loads in flight while
-      // this chunk is combined and stored
+      // old values of the chunks past the first two of the first half: the
+      // next chunk's loads in flight while this chunk is combined and stored
       float4 ov[8];
       auto load_old = [&](int c0) {
         if (mine && !ud.init)
 #pragma unroll
           for (int q = 0; q < 8; ++q) ov[q] = g4[c0 / 4 + q];
       };
-      load_old(dlo);
-#pragma unroll 1
-      for (int c0 = dlo; c0 < dhi; c0 += 32) {
+      if (hh > 0) load_old(dlo);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (k >= nchunk) break;
+        const int c0 = dlo + 32 * k;
+        const bool early = hh == 0 && k < 2;  // loaded before the tiles
         float sm[32];
         tmem_ld32(tmem_base + lane_addr + acol + 128u * hh + c0, sm);  // warp-collective
         float v[32];
@@ -286,11 +302,12 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
           } else {
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-              v[4 * q] = ov[q].x; v[4 * q + 1] = ov[q].y; v[4 * q + 2] = ov[q].z; v[4 * q + 3] = ov[q].w;
+              const float4 o = early ? ov0[8 * (k & 1) + q] : ov[q];
+              v[4 * q] = o.x; v[4 * q + 1] = o.y; v[4 * q + 2] = o.z; v[4 * q + 3] = o.w;
             }
           }
         }
-        if (c0 + 32 < dhi) load_old(c0 + 32);
+        if (k + 1 < nchunk && !(hh == 0 && k + 1 < 2)) load_old(c0 + 32);
         if (mine) {
           if (m > 0)
 #pragma unroll
