@@ -115,17 +115,26 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
   for (int i = tid; i < 32768 / 16; i += kUT) reinterpret_cast<uint4 *>(asum)[i] = make_uint4(0, 0, 0, 0);
   for (int b = tid; b < B; b += kUT) cnt[b] = 0;
   // beacons: bf16 hi/lo terms in the swizzled layout, fp32 squared norms;
-  // 32 beacons' loads in flight at once
-  for (int b0 = 0; b0 < B; b0 += 32) {  // B is a multiple of 32
-    float c[32];
+  // 32 beacons' loads in flight at once, the next 32 issued before this
+  // batch is split and stored
+  float cnext[32];
+  auto load_batch = [&](int b0) {
     if (ud.init) {
 #pragma unroll
-      for (int u = 0; u < 32; ++u) c[u] = c_old(b0 + u, tid);
+      for (int u = 0; u < 32; ++u) cnext[u] = c_old(b0 + u, tid);
     } else {
       // no branch between the loads, so all 32 are in flight together
 #pragma unroll
-      for (int u = 0; u < 32; ++u) c[u] = gbeac[(b0 + u) * D + tid];
+      for (int u = 0; u < 32; ++u) cnext[u] = gbeac[(b0 + u) * D + tid];
     }
+  };
+  load_batch(0);
+#pragma unroll 1
+  for (int b0 = 0; b0 < B; b0 += 32) {  // B is a multiple of 32
+    float c[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) c[u] = cnext[u];
+    if (b0 + 32 < B) load_batch(b0 + 32);
     const int kb = tid >> 6, k = tid & 63;
 #pragma unroll
     for (int u8 = 0; u8 < 32; u8 += 8) {
