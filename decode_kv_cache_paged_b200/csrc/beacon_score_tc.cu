@@ -21,11 +21,14 @@
 //          and takes the max over beacon columns of u_bj - lse2_b.
 // Work in base 2: u = z_raw * log2(e)/sqrt(d), lse2 = log2 sum 2^u, score =
 // 2^(max_b u_bj - lse2_b).
-// Warp roles: warp 0 allocates TMEM and issues the TMA loads (one 2-D tiled
-// load per (page, 64-column half), lane q of the warp taking page q of the
-// tile, page ids loaded one tile ahead: a page holds 16 keys x 256 B contiguous,
-// the tensor map covers the whole pool as rows of 128 bf16, 128-byte
-// swizzle); warp 1 issues the MMAs (one elected lane) and commits them to
+// Warp roles: warp 0 allocates TMEM and issues the TMA loads (128-byte
+// swizzle, page ids loaded one tile ahead): a tile whose 8 page ids are
+// consecutive comes in as two 4-D boxes (64 columns x 16 rows x 8 pages of
+// one head, the pool seen as columns, rows, heads, layer * pages); any other
+// tile as one 2-D box per (page, 64-column half), lane q of the warp taking
+// page q (a page holds 16 keys x 256 B contiguous; that map covers the pool
+// as rows of 128 bf16).  The number of boxes, not their bytes, limited the
+// key stream; warp 1 issues the MMAs (one elected lane) and commits them to
 // mbarriers; warps 2-9 run the epilogue in two groups of four, group g taking
 // the tiles whose accumulator is in TMEM buffers of parity g (tcgen05.ld of
 // 64 columns at a time; sums and maxima in 8 independent partials; the
@@ -106,10 +109,22 @@ __device__ __forceinline__ SegGeom seg_geom(const TcParams &p, int s) {
   return g;
 }
 
+// 4-D tiled load (no multicast): the key pool seen as (128 columns, 16 rows,
+// KV heads, layer * pages + page), so one box brings the same 64 columns of 8
+// consecutive page ids' 16 rows of one head
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int x, int y, int z, int w,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
 template <int CROWS, int NCB, int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
     beacon_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap cmap,
-                           TcParams p) {
+                           const __grid_constant__ CUtensorMap kmap4, TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_align<1024>(smem_raw);
   constexpr uint32_t kCBytes = CROWS * 256;          // beacon tile: CROWS rows x 128 bf16
@@ -214,7 +229,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int npg = min(kTP, pages - tile * kTP);
           if (lane == 0) mbar_expect_tx(&full[st], (uint32_t)npg * 2u * 2048u);
           __syncwarp();
-          if (lane < npg) {
+          // a full tile whose 8 page ids are consecutive: two 4-D boxes (8
+          // pages x 16 rows x 64 columns, the same 16 KB layout) instead of
+          // 16 page boxes
+          const int pg_first = __shfl_sync(0xffffffffu, pg_cur, 0);
+          const bool run = npg == kTP && __all_sync(0xffffffffu, lane >= kTP || pg_cur == pg_first + lane);
+          if (run) {
+            if (lane < 2)
+              tma_load_4d(smem_u32(kbuf + st * kTileBytes + lane * kTileKeys * 128), &kmap4, lane * 64, 0, g.h,
+                          (int)(g.l * p.num_pages) + pg_first, &full[st]);
+          } else if (lane < npg) {
             uint8_t *dst = kbuf + st * kTileBytes;
             const int64_t row = (((int64_t)g.l * p.num_pages + pg_cur) * p.hkv + g.h) * kPage;
             tma_load_2d(smem_u32(dst + lane * 2048), &kmap, 0, (int)row, &full[st]);
@@ -504,8 +528,23 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// the same pool as (128 columns, 16 rows, hkv heads, layers * pages), box
+// (64 columns, 16 rows, 1 head, 8 pages), 128-byte swizzle
+bool make_map4(CUtensorMap *m, const void *base, uint64_t layer_pages, uint32_t hkv) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {128, kPage, hkv, layer_pages};
+  cuuint64_t strides[3] = {256, (cuuint64_t)kPage * 256, (cuuint64_t)hkv * kPage * 256};
+  cuuint32_t box[4] = {64, kPage, 1, kTileKeys / kPage};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int CROWS, int NCB, int kStages>
-cudaError_t launch(const CUtensorMap &km, const CUtensorMap &cm, const TcParams &tp, cudaStream_t s) {
+cudaError_t launch(const CUtensorMap &km, const CUtensorMap &cm, const CUtensorMap &km4, const TcParams &tp,
+                   cudaStream_t s) {
   const size_t smem = 1024 + (size_t)NCB * CROWS * 256 + (size_t)kStages * kTileKeys * 256 + 256 +
                       2 * 256 * 4 + 4 * 2 * 256 * 4 + 2 * 256 * 4;
   cudaError_t e = cudaFuncSetAttribute(beacon_score_tc_kernel<CROWS, NCB, kStages>,
@@ -515,7 +554,7 @@ cudaError_t launch(const CUtensorMap &km, const CUtensorMap &cm, const TcParams 
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = tp.n_segs < sms ? tp.n_segs : sms;
-  beacon_score_tc_kernel<CROWS, NCB, kStages><<<grid, kThreads, smem, s>>>(km, cm, tp);
+  beacon_score_tc_kernel<CROWS, NCB, kStages><<<grid, kThreads, smem, s>>>(km, cm, km4, tp);
   return cudaGetLastError();
 }
 
@@ -529,12 +568,13 @@ cudaError_t launch_beacon_score_tc(const BeaconScoreParams &p, int n_req, int ma
   (void)max_l;
   if (!beacon_score_tc_supported(p.d, p.B, p.dtype)) return cudaErrorNotSupported;
   if (n_req <= 0) return cudaSuccess;
-  CUtensorMap km, cm;
+  CUtensorMap km, cm, km4;
   const uint64_t krows = (uint64_t)p.layers * (uint64_t)p.num_pages * (uint64_t)p.hkv * kPage;
   // the beacon map spans every (request, layer, head) segment's B rows
   const uint64_t crows = (uint64_t)p.total_segs * (uint64_t)p.B;
   if (krows >= (1ull << 31) || crows >= (1ull << 31)) return cudaErrorInvalidValue;
-  if (!make_map(&km, p.k_pool, krows, kPage) || !make_map(&cm, p.beacons_s, crows, (uint32_t)p.B))
+  if (!make_map(&km, p.k_pool, krows, kPage) || !make_map(&cm, p.beacons_s, crows, (uint32_t)p.B) ||
+      !make_map4(&km4, p.k_pool, (uint64_t)p.layers * (uint64_t)p.num_pages, (uint32_t)p.hkv))
     return cudaErrorInvalidValue;
   TcParams tp{};
   tp.block_table = p.block_table;
@@ -551,8 +591,8 @@ cudaError_t launch_beacon_score_tc(const BeaconScoreParams &p, int n_req, int ma
   tp.max_seq = p.max_seq;
   tp.n_segs = n_req * p.layers * p.hkv;
   tp.alpha = 1.4426950408889634f / sqrtf(128.0f);
-  if (p.B <= 128) return launch<128, KVC_TC_NCB_SMALL, KVC_TC_STAGES_SMALL>(km, cm, tp, s);
-  return launch<256, 1, 4>(km, cm, tp, s);
+  if (p.B <= 128) return launch<128, KVC_TC_NCB_SMALL, KVC_TC_STAGES_SMALL>(km, cm, km4, tp, s);
+  return launch<256, 1, 4>(km, cm, km4, tp, s);
 }
 
 }  // namespace kvc

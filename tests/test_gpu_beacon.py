@@ -17,40 +17,50 @@ from gpu_helpers import band_check, check_scores, dense_layer, make_context
 pytestmark = pytest.mark.gpu
 
 
-def _fill_recording(ctx, w, gen):
-    """Fill like workloads.fill, keeping the queries of the last W steps per request."""
+def _fill_recording(ctx, w, gen, interleave=False):
+    """Fill like workloads.fill, keeping the queries of the last W steps per request.  With interleave, the
+    requests take turns appending 16 tokens (one page) at a time, so no request holds consecutive page ids."""
     R = w.num_requests
     W = w.query_window
-    qwin = {}
+    plans = []
     for r in range(R):
         P, L = int(w.prompt[r]), int(w.length[r])
-        ids = np.array([r], np.int32)
-        done = 0
-        while done < P:
-            T = min(256, P - done)
-            k, v = gen.kv(1, T)
-            ctx.append(ids, k, v, None, protect=True)
-            done += T
         q_from = L - min(W, L - P)
-        qs = []
-        while done < L:
-            T = min(256 if done < q_from else 16, (q_from if done < q_from else L) - done)
-            k, v = gen.kv(1, T)
-            q = gen.queries(1, T) if done >= q_from else None
-            ctx.append(ids, k, v, q)
-            if q is not None:
-                qs.append(q[0].float().cpu().numpy().astype(np.float64))  # [Ly, T, Hq, d]
+        steps, done = [], 0  # (tokens, protect, with queries)
+        while done < P:
+            T = min(16 if interleave else 256, P - done)
+            steps.append((T, True, False))
             done += T
-        qwin[r] = np.concatenate(qs, axis=1)[:, -W:]  # [Ly, steps, Hq, d]
-    return qwin
+        while done < L:
+            T = min(256 if done < q_from and not interleave else 16, (q_from if done < q_from else L) - done)
+            steps.append((T, False, done >= q_from))
+            done += T
+        plans.append(steps)
+    if interleave:
+        order = [(r, plans[r][i]) for i in range(max(len(pl) for pl in plans)) for r in range(R) if i < len(plans[r])]
+    else:
+        order = [(r, st) for r in range(R) for st in plans[r]]
+    qs = {r: [] for r in range(R)}
+    for r, (T, protect, with_q) in order:
+        ids = np.array([r], np.int32)
+        k, v = gen.kv(1, T)
+        if protect:
+            ctx.append(ids, k, v, None, protect=True)
+            continue
+        q = gen.queries(1, T) if with_q else None
+        ctx.append(ids, k, v, q)
+        if q is not None:
+            qs[r].append(q[0].float().cpu().numpy().astype(np.float64))  # [Ly, T, Hq, d]
+    return {r: np.concatenate(qs[r], axis=1)[:, -W:] for r in range(R)}  # [Ly, steps, Hq, d]
 
 
-def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered", selector="beacon", k_hook=None):
+def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered", selector="beacon", k_hook=None,
+               interleave=False):
     ctx = make_context(w)
     if score_impl is not None:
         ctx.set_option(0, score_impl)
     gen = wl.Generator(w, "cuda")
-    qwin = _fill_recording(ctx, w, gen)
+    qwin = _fill_recording(ctx, w, gen, interleave)
     R, Ly, H, d, B, G = w.num_requests, w.num_layers, w.num_kv_heads, w.head_dim, w.num_beacons, w.G
     W = w.query_window
     assign = torch.full((R, Ly, H, W * G), -1, dtype=torch.int32, device="cuda")
@@ -230,6 +240,14 @@ def test_tcgen05_256_beacons():
     w.budget = np.array([1000])
     w.prompt = np.array([77])
     out = run_beacon(w, score_impl=2)
+    print(out)
+
+
+def test_tcgen05_scattered_pages():
+    """Two requests filled one page at a time in turn: no 8-page key tile has consecutive page ids, so every
+    tile comes in as per-page boxes (with consecutive ids a tile is two 8-page boxes)."""
+    w = wl.beacon_serving(R=2, layers=2)
+    out = run_beacon(w, score_impl=2, interleave=True)
     print(out)
 
 
