@@ -194,6 +194,30 @@ def profiled_traffic(kernel: str, workload: str, units: float):
     return e["dram_bytes_per_unit"] * units
 
 
+def score_roofline(flops: float, nbytes: float, ms: float, peaks: dict, clocks, tensor_cores: bool) -> dict:
+    """Roofline entry of the beacon score kernel.  The tcgen05 kernel is HBM-bound
+    when its flops per algorithmic byte fall below the ridge (tensor peak / HBM
+    peak), tensor-bound otherwise; the tensor peak is the sustained (power-capped)
+    figure when the sampled clocks saw the cap, else the burst one.  The SIMT
+    kernel is held against the fp32 pipe: 148 SMs x 128 lanes x 2 flop x the max
+    SM clock."""
+    sec = ms / 1e3
+    if tensor_cores:
+        capped = "sw_power_cap" in (clocks or {}).get("reasons", [])
+        tpeak = peaks.get("bf16_tflops_sustained" if capped else "bf16_tflops")
+        ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        if flops / nbytes < ridge:
+            return {"kernel": "beacon_score_tc", "bound": "hbm", "achieved": nbytes / sec / 1e9,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "tflops": flops / sec / 1e12,
+                    "flop_per_byte": flops / nbytes}
+        return {"kernel": "beacon_score_tc", "bound": "tensor", "achieved": flops / sec / 1e12, "peak": tpeak,
+                "unit": "TFLOP/s", "peak_kind": "sustained" if capped else "burst", "hbm_gbs": nbytes / sec / 1e9,
+                "flop_per_byte": flops / nbytes}
+    simt_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    return {"kernel": "beacon_score_simt", "bound": "alu", "achieved": flops / sec / 1e12, "peak": simt_peak,
+            "unit": "TFLOP/s", "hbm_gbs": nbytes / sec / 1e9}
+
+
 # ------------------------------------------------------------ our arm ---
 
 def aggregate(local_ms: float, units_per_rank: float, steps: int, world: int, dist, device=None):
@@ -339,25 +363,7 @@ def run_ours(args, rank, world, dist):
         keys = key_bytes / rb
         flops = 2.0 * B * w.head_dim * (keys + cands)  # pass 1 over all keys, pass 2 over candidates
         score_bytes = key_bytes + cands * 4 + (w.segments * B * w.head_dim * (2 if w.dtype == "bf16" else 4))
-        tc = stats[-1].get("score_kernel", 0) == 2
-        # the tensor peak that matches the clocks seen while timing: sustained
-        # (power-capped) when the cap was active, else the burst figure
-        capped = "sw_power_cap" in (clocks or {}).get("reasons", [])
-        tpeak = peaks.get("bf16_tflops_sustained" if capped else "bf16_tflops")
-        ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)  # flop per byte where the bounds meet
-        if tc and flops / score_bytes < ridge:
-            roof = {"kernel": "beacon_score_tc", "bound": "hbm", "achieved": score_bytes / (score_ms / 1e3) / 1e9,
-                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "tflops": flops / (score_ms / 1e3) / 1e12, "flop_per_byte": flops / score_bytes}
-        elif tc:
-            roof = {"kernel": "beacon_score_tc", "bound": "tensor", "achieved": flops / (score_ms / 1e3) / 1e12,
-                    "peak": tpeak, "unit": "TFLOP/s", "peak_kind": "sustained" if capped else "burst",
-                    "hbm_gbs": score_bytes / (score_ms / 1e3) / 1e9, "flop_per_byte": flops / score_bytes}
-        else:
-            # SIMT fp32: 148 SMs x 128 FP32 lanes x 2 flop per FMA x the max SM clock
-            simt_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-            roof = {"kernel": "beacon_score_simt", "bound": "alu", "achieved": flops / (score_ms / 1e3) / 1e12,
-                    "peak": simt_peak, "unit": "TFLOP/s", "hbm_gbs": score_bytes / (score_ms / 1e3) / 1e9}
+        roof = score_roofline(flops, score_bytes, score_ms, peaks, clocks, stats[-1].get("score_kernel", 0) == 2)
         roof["traffic"] = profiled_traffic(roof["kernel"], w.name, keys)
     else:
         roof = {"kernel": "select_compact", "bound": "hbm", "achieved": sc_bytes / (sc_ms / 1e3) / 1e9,
@@ -365,7 +371,9 @@ def run_ours(args, rank, world, dist):
                 "traffic": profiled_traffic("select_compact", traffic_key, moved)}
     roof["frac"] = roof["achieved"] / roof["peak"] if roof.get("peak") else None
     roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})"
-    roof["algorithmic_bytes_per_launch"] = sc_bytes if roof["kernel"] == "select_compact" else None
+    roof["algorithmic_bytes_per_launch"] = sc_bytes if roof["kernel"] == "select_compact" else score_bytes
+    if roof["kernel"] != "select_compact":
+        roof["algorithmic_flops_per_launch"] = flops
     roof["launch_ms"] = sc_ms if roof["kernel"] == "select_compact" else score_ms
 
     # end to end through the public API, every step: the next trigger window's

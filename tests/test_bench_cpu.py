@@ -1,0 +1,68 @@
+"""bench.py's roofline bookkeeping on the CPU: the score kernel's bound and
+peak choice, and the traffic lookup gated by the kernel sources' hash."""
+import json
+import os
+
+import pytest
+
+import bench
+
+PEAKS = {"hbm_gbs": 6529.4, "bf16_tflops": 1674.6, "bf16_tflops_sustained": 1388.6, "sm_max_mhz": 1965.0}
+
+
+def test_score_roofline_hbm_below_ridge():
+    # 64 flop per byte is under both ridges (256 burst, 213 sustained)
+    r = bench.score_roofline(64e12, 1e12, 1000.0, PEAKS, {"reasons": []}, True)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(1000.0) and r["peak"] == PEAKS["hbm_gbs"]
+    assert r["flop_per_byte"] == pytest.approx(64.0)
+
+
+@pytest.mark.parametrize("reasons,peak,kind", [([], 1674.6, "burst"), (["sw_power_cap"], 1388.6, "sustained")])
+def test_score_roofline_tensor_above_ridge(reasons, peak, kind):
+    r = bench.score_roofline(500e12, 1e12, 1000.0, PEAKS, {"reasons": reasons}, True)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["peak"] == peak and r["peak_kind"] == kind
+    assert r["achieved"] == pytest.approx(500.0)
+
+
+def test_score_roofline_ridge_follows_the_peak():
+    # 230 flop per byte: tensor-bound against the sustained ridge (213), HBM-bound against the burst one (256)
+    assert bench.score_roofline(230e12, 1e12, 1.0, PEAKS, {"reasons": ["sw_power_cap"]}, True)["bound"] == "tensor"
+    assert bench.score_roofline(230e12, 1e12, 1.0, PEAKS, {"reasons": []}, True)["bound"] == "hbm"
+
+
+def test_score_roofline_simt():
+    r = bench.score_roofline(74.4e12, 1e12, 1000.0, PEAKS, None, False)
+    assert r["bound"] == "alu" and r["kernel"] == "beacon_score_simt"
+    assert r["peak"] == pytest.approx(148 * 128 * 2 * 1965e6 / 1e12)
+
+
+def test_traffic_lookup_gated_by_source_hash(tmp_path, monkeypatch):
+    src = ["select_compact.cu", "philox.cuh"]
+    good = {"sources": src, "source_hash": bench.kernel_source_hash(src), "unit": "moved row",
+            "dram_bytes_per_unit": 1000.0}
+    stale = dict(good, source_hash="0" * 16)
+    path = tmp_path / "traffic.json"
+    path.write_text(json.dumps({"select_compact": {"a": good, "b": stale}}))
+    monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(path))
+    assert bench.profiled_traffic("select_compact", "a", 3.0) == pytest.approx(3000.0)
+    assert bench.profiled_traffic("select_compact", "b", 3.0) is None
+    assert bench.profiled_traffic("select_compact", "missing", 3.0) is None
+    assert bench.profiled_traffic("decode_attention", "a", 3.0) is None
+
+
+def test_committed_traffic_entries_are_well_formed():
+    with open(bench.PROFILE_TRAFFIC) as f:
+        t = json.load(f)
+    csrc = os.path.join(bench.ROOT, "decode_kv_cache_paged_b200", "csrc")
+    n = 0
+    for kernel, entries in t.items():
+        if kernel == "about":
+            continue
+        for workload, e in entries.items():
+            assert e["dram_bytes_per_unit"] > 0 and e["unit"] and e["captured"], (kernel, workload)
+            assert all(os.path.exists(os.path.join(csrc, s)) for s in e["sources"]), (kernel, workload)
+            assert len(e["source_hash"]) == 16
+            n += 1
+    assert n >= 4
