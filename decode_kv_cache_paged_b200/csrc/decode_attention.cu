@@ -27,7 +27,9 @@
 //     K rows themselves, a quarter-warp reading 128 consecutive bytes.  The
 //     lanes of a row then sum their partial dot products with a butterfly
 //     reduce-scatter (each exchange halves the sums a lane holds), ending
-//     with each lane holding whole scores of one row for a few heads.  The
+//     with each lane holding whole scores of one row for a few heads; each
+//     lane stores its partial sums in a lane-dependent order so that the
+//     exchanges need no selects.  The
 //     query used to be re-read from shared memory for every chunk, which
 //     made the shared-memory data pipe the limit.  Online softmax in base 2
 //     with the scale folded into q.
@@ -129,29 +131,28 @@ struct AttnShape {
 };
 
 // Reduce-scatter of N partial sums over the lanes xor M, M/2, ..., 1 apart:
-// each exchange sends half of the sums still held to the partner and adds
-// the partner's half of its own; once a lane holds one sum the remaining
-// exchanges add the partner's copy of it.  Afterwards, with M = the lanes of
-// a row / 2, lane c of the row holds the whole sums of entries
-// c * N / (2M) + k, k < max(1, N / (2M)), in v[k].
+// each exchange keeps the lower half of the sums still held and adds the
+// partner's upper half; once a lane holds one sum the remaining exchanges add
+// the partner's copy of it.  The lanes store their partial sums permuted (see
+// the kernel) so that at every exchange the lower half holds the entries this
+// lane keeps and the upper half those its partner keeps: no selects.
+// Afterwards, with M = the lanes of a row / 2, lane c of the row holds the
+// whole sums of entries c * N / (2M) + k, k < max(1, N / (2M)), in v[k].
 template <int N, int M, int NV>
-__device__ __forceinline__ void reduce_scatter(float (&v)[NV], int lane) {
+__device__ __forceinline__ void reduce_scatter(float (&v)[NV]) {
   if constexpr (M >= 1) {
     if constexpr (N > 1) {
-      const bool upper = (lane & M) != 0;
 #pragma unroll
-      for (int k = 0; k < N / 2; ++k) {
-        const float send = upper ? v[k] : v[k + N / 2];
-        const float keep = upper ? v[k + N / 2] : v[k];
-        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, M);
-      }
-      reduce_scatter<N / 2, M / 2>(v, lane);
+      for (int k = 0; k < N / 2; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k + N / 2], M);
+      reduce_scatter<N / 2, M / 2>(v);
     } else {
       v[0] += __shfl_xor_sync(0xffffffffu, v[0], M);
-      reduce_scatter<1, M / 2>(v, lane);
+      reduce_scatter<1, M / 2>(v);
     }
   }
 }
+
+constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 
 // Each of the 4 warps walks every 4th page of the CTA's split through its own
 // 2-slot ring (K and V of one page per slot), with its own running max and
@@ -216,16 +217,32 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(DecodeAttnPa
   const int g0 = e0 % G;
   const bool writer = (c % S::kDup) == 0;  // one lane of each set of copies stores
 
-  // chunk c of this KV head's G query rows, scaled into base 2, in registers
+  // The lane stores partial sum (i, g) of a batch in slot (i ^ p_row, g ^
+  // p_head): its lane bit of the exchange at mask kLpr/2 >> st flips slot bit
+  // log2(kNv) - 1 - st, for the exchanges that split.  Then at every exchange
+  // the entries this lane keeps sit in the lower half of its array and the
+  // ones its partner keeps in the upper half.
+  int perm = 0;
+  {
+    constexpr int kLogNv = ilog2(S::kNv), kSplit = ilog2(S::kLpr) < kLogNv ? ilog2(S::kLpr) : kLogNv;
+#pragma unroll
+    for (int st = 0; st < kSplit; ++st)
+      if (lane & ((S::kLpr / 2) >> st)) perm |= 1 << (kLogNv - 1 - st);
+  }
+  const int p_row = perm >> ilog2(G), p_head = perm & (G - 1);
+
+  // chunk c of this KV head's G query rows (head g ^ p_head in slot g), scaled
+  // into base 2, in registers
   float2 qr[G][S::kPairs];
   {
     const T *q = reinterpret_cast<const T *>(p.q) + (((int64_t)lc * p.R + r) * p.hq + (int64_t)h * G) * D;
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+    for (int g = 0; g < G; ++g) {
+      const T *qg = q + (g ^ p_head) * D + c * S::kEpc;
 #pragma unroll
       for (int e = 0; e < S::kPairs; ++e)
-        qr[g][e] = make_float2(to_float(q[g * D + c * S::kEpc + 2 * e]) * p.qscale,
-                               to_float(q[g * D + c * S::kEpc + 2 * e + 1]) * p.qscale);
+        qr[g][e] = make_float2(to_float(qg[2 * e]) * p.qscale, to_float(qg[2 * e + 1]) * p.qscale);
+    }
   }
 
   float m_run[KEEP], l_lane[KEEP];
@@ -256,10 +273,10 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(DecodeAttnPa
     float sv[S::kBatches][KEEP];
 #pragma unroll
     for (int b = 0; b < S::kBatches; ++b) {
-      float part[S::kNv];  // entry i * G + g: row i of the batch, head g
+      float part[S::kNv];  // slot i * G + g: row i ^ p_row of the batch, head g ^ p_head
 #pragma unroll
       for (int i = 0; i < S::kRb; ++i) {
-        const int row = grp * S::kRowsPerGroup + b * S::kRb + i;
+        const int row = grp * S::kRowsPerGroup + b * S::kRb + (i ^ p_row);
         float2 x[S::kPairs];
         load_chunk2<T>(kp + row * S::kRowBytes + c * 16, x);
 #pragma unroll
@@ -270,7 +287,7 @@ __global__ void __launch_bounds__(kThreads) decode_attention_kernel(DecodeAttnPa
           part[i * G + g] = t.x + t.y;
         }
       }
-      reduce_scatter<S::kNv, S::kLpr / 2>(part, lane);
+      reduce_scatter<S::kNv, S::kLpr / 2>(part);
       const int row = grp * S::kRowsPerGroup + b * S::kRb + e0 / G;
 #pragma unroll
       for (int kk = 0; kk < KEEP; ++kk) sv[b][kk] = row < valid ? part[kk] : -INFINITY;
