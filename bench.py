@@ -2,7 +2,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload random_serving|beacon_serving|long_trace|ragged_c2|...]
-                    [--requests R] [--layers L] [--no-cpu-baseline] [--no-e2e]
+                    [--extras beacon_serving,long_trace,ragged_c2] [--extra-steps K2]
+                    [--requests R] [--layers L] [--no-cpu-baseline] [--no-cpu-pool] [--no-e2e]
 
 A step is one eviction round (kvc_update_beacons + kvc_compress for the
 beacon selector, kvc_compress for the random ones) over every (request,
@@ -14,10 +15,15 @@ Random Attention article's serving setup ("发现四": K=2048, 1k-token prompt,
 
 Printed (rank 0, one JSON line): head-positions compressed per second over the
 K timed rounds (device time, CUDA events on the library's stream; max over
-ranks for N > 1), the roofline of the dominant kernel, the CPU oracle timed
-on a bounded sample (cpu_baseline), an end-to-end figure through the C ABI
-with the trigger window's K/V (and queries) read from page-locked host
-memory every step, and the clocks sampled during the timed region.
+ranks for N > 1), the roofline of the dominant kernel and of every kernel of
+the round, the CPU oracle timed on bounded samples on one host core
+(cpu_baseline) and on all of them (cpu_baseline_all_cores), an end-to-end
+figure through the C ABI with the trigger window's K/V (and queries) read
+from page-locked host memory every step, and the clocks sampled during the
+timed region.  The headline workload is the random serving round; the
+BeaconKV serving round, the long-trace compression and the ragged sweep's
+2x slice follow with fewer rounds each, under extra_workloads, each with its
+own phases, rooflines, clocks and CPU baselines.
 
 Multi-GPU: one process per GPU (torchrun), each rank an independent replica
 with its own requests (the round has no exchange step: weak scaling, no
@@ -55,8 +61,12 @@ def parse():
     ap.add_argument("--requests", type=int, default=None)
     ap.add_argument("--layers", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-pool", action="store_true",
-                    help="also time the oracle over all host cores (one spawned process per core)")
+    ap.add_argument("--no-cpu-pool", action="store_true",
+                    help="skip timing the oracle over all host cores (one spawned process per core)")
+    ap.add_argument("--extras", default="beacon_serving,long_trace,ragged_c2",
+                    help="comma-separated workloads also timed (fewer rounds) after the headline one and "
+                         "reported under extra_workloads; '' for none")
+    ap.add_argument("--extra-steps", type=int, default=8, help="timed rounds of each extra workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--score-impl", type=int, default=0, help="beacon score kernel: 0 auto, 1 SIMT, 2 tcgen05")
@@ -194,28 +204,59 @@ def profiled_traffic(kernel: str, workload: str, units: float):
     return e["dram_bytes_per_unit"] * units
 
 
-def score_roofline(flops: float, nbytes: float, ms: float, peaks: dict, clocks, tensor_cores: bool) -> dict:
-    """Roofline entry of the beacon score kernel.  The tcgen05 kernel is HBM-bound
-    when its flops per algorithmic byte fall below the ridge (tensor peak / HBM
-    peak), tensor-bound otherwise; the tensor peak is the sustained (power-capped)
-    figure when the sampled clocks saw the cap, else the burst one.  The SIMT
-    kernel is held against the fp32 pipe: 148 SMs x 128 lanes x 2 flop x the max
-    SM clock."""
+def score_roofline(flops: float, nbytes: float, ms: float, peaks: dict, tensor_cores: bool,
+                   recompute_flops: float = 0.0) -> dict:
+    """Roofline entry of the beacon score kernel.
+
+    flops is the method's work: one product of 2*d flops per (beacon, cached
+    key) pair.  The two-pass log-sum-exp computes the candidates' products a
+    second time; those recompute_flops are reported beside it but are not
+    algorithmic work, so they show up as a lower fraction.  The kernel is timed
+    on its own by CUDA events around its launch, so the tensor peak is the
+    burst figure.  The tcgen05 kernel is HBM-bound when its flops per
+    algorithmic byte fall below the ridge (tensor peak / HBM peak),
+    tensor-bound otherwise.  The SIMT kernel is held against the fp32 pipe:
+    148 SMs x 128 lanes x 2 flop x the max SM clock."""
     sec = ms / 1e3
+    extra = {"algorithmic_flops_per_launch": flops, "recompute_flops_per_launch": recompute_flops,
+             "executed_tflops": (flops + recompute_flops) / sec / 1e12, "flop_per_byte": flops / nbytes,
+             "algorithmic_bytes_per_launch": nbytes, "launch_ms": ms}
     if tensor_cores:
-        capped = "sw_power_cap" in (clocks or {}).get("reasons", [])
-        tpeak = peaks.get("bf16_tflops_sustained" if capped else "bf16_tflops")
+        tpeak = peaks.get("bf16_tflops")
         ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        hbm = {"hbm_gbs": nbytes / sec / 1e9, "hbm_frac": nbytes / sec / 1e9 / peaks["hbm_gbs"]}
+        ten = {"tflops": flops / sec / 1e12, "tensor_frac": flops / sec / 1e12 / tpeak, "tensor_peak": tpeak,
+               "peak_kind": "burst", "ridge_flop_per_byte": ridge}
         if flops / nbytes < ridge:
-            return {"kernel": "beacon_score_tc", "bound": "hbm", "achieved": nbytes / sec / 1e9,
-                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "tflops": flops / sec / 1e12,
-                    "flop_per_byte": flops / nbytes}
-        return {"kernel": "beacon_score_tc", "bound": "tensor", "achieved": flops / sec / 1e12, "peak": tpeak,
-                "unit": "TFLOP/s", "peak_kind": "sustained" if capped else "burst", "hbm_gbs": nbytes / sec / 1e9,
-                "flop_per_byte": flops / nbytes}
-    simt_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-    return {"kernel": "beacon_score_simt", "bound": "alu", "achieved": flops / sec / 1e12, "peak": simt_peak,
-            "unit": "TFLOP/s", "hbm_gbs": nbytes / sec / 1e9}
+            out = {"kernel": "beacon_score_tc", "bound": "hbm", "achieved": nbytes / sec / 1e9,
+                   "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        else:
+            out = {"kernel": "beacon_score_tc", "bound": "tensor", "achieved": flops / sec / 1e12, "peak": tpeak,
+                   "unit": "TFLOP/s"}
+        out.update(hbm)
+        out.update(ten)
+    else:
+        simt_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        out = {"kernel": "beacon_score_simt", "bound": "alu", "achieved": flops / sec / 1e12, "peak": simt_peak,
+               "unit": "TFLOP/s", "hbm_gbs": nbytes / sec / 1e9}
+    out.update(extra)
+    return out
+
+
+def update_roofline(w, ms: float, peaks: dict, tensor_cores: bool) -> dict:
+    """Roofline entry of the beacon update: per segment the window's points
+    (W steps x G query heads x d) are read once, and the fp32 beacons are read
+    and written, their scoring copy written and the counts and trigger shares
+    read and written once.  HBM-bound by its bytes (a few flops per byte)."""
+    es = 2 if w.dtype == "bf16" else 4
+    B, d = w.num_beacons, w.head_dim
+    per_seg = w.query_window * w.G * d * es + B * d * (4 + 4 + es) + B * (4 + 4 + 4)
+    nbytes = w.segments * per_seg
+    sec = ms / 1e3
+    return {"kernel": "beacon_update_tc" if tensor_cores else "beacon_update_simt", "bound": "hbm",
+            "achieved": nbytes / sec / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": nbytes / sec / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes,
+            "launch_ms": ms, "traffic": None}
 
 
 # ------------------------------------------------------------ our arm ---
@@ -272,7 +313,53 @@ class Refill:
                 ctx.append(ids, k, v, q)
                 done += T
 
-def run_ours(args, rank, world, dist):
+def round_rooflines(w, sel, stats, upd_ms, peaks, args) -> dict:
+    """Roofline entries of every kernel of the round, from the timed rounds'
+    own counters: select_compact always, the score and update kernels under
+    the beacon selectors."""
+    beacon = sel in ("beacon", "beacon_trigger")
+    variant = [] if args.compaction == "ordered" else [args.compaction]
+    variant += [f"block{args.block}"] if args.block != 1 else []
+    variant += [f"sinks{args.sinks}"] if args.sinks is not None else []
+    traffic_key = "/".join([w.name] + variant)
+    sc_ms = statistics.mean(s["ms_select_compact"] for s in stats)
+    moved = statistics.mean(s["moved_rows"] for s in stats)
+    cands = statistics.mean(s["candidates"] for s in stats)
+    es = 2 if w.dtype == "bf16" else 4
+    rb = w.head_dim * es
+    # select+compact: K and V rows read and written once per moved row, the moved
+    # position entries read and written, every candidate's 4-byte key source read
+    sc_bytes = moved * (4 * rb + 8) + cands * 4
+    peak_src = "MEASURED_PEAKS.json" if peaks.get("_kind") == "measured" else "recipe fallback"
+    out = {"select_compact": {
+        "kernel": "select_compact", "bound": "hbm", "achieved": sc_bytes / (sc_ms / 1e3) / 1e9,
+        "peak": peaks["hbm_gbs"], "unit": "GB/s", "traffic": profiled_traffic("select_compact", traffic_key, moved),
+        "algorithmic_bytes_per_launch": sc_bytes, "launch_ms": sc_ms, "moved_rows": moved, "candidates": cands}}
+    if beacon:
+        score_ms = statistics.mean(s["ms_score"] for s in stats)
+        key_bytes = statistics.mean(s["key_bytes_scored"] for s in stats)
+        keys = key_bytes / rb
+        B = w.num_beacons
+        flops = 2.0 * B * w.head_dim * keys          # one product per (beacon, cached key) pair
+        recompute = 2.0 * B * w.head_dim * cands     # pass 2 recomputes the candidates' products
+        score_bytes = key_bytes + cands * 4 + w.segments * B * rb
+        tc = stats[-1].get("score_kernel", 0) == 2
+        roof = score_roofline(flops, score_bytes, score_ms, peaks, tc, recompute)
+        roof["traffic"] = profiled_traffic(roof["kernel"], w.name, keys)
+        out["score"] = roof
+        upd = statistics.mean(upd_ms)
+        out["update"] = update_roofline(w, upd, peaks, w.dtype == "bf16" and w.head_dim == 128)
+    for r in out.values():
+        r["frac"] = r["achieved"] / r["peak"] if r.get("peak") else None
+        r["peak_source"] = f"{peaks.get('_kind')} ({peak_src})"
+    return out
+
+
+def run_ours(args, rank, world, dist, with_e2e=True):
+    """One workload: fill, W warm-up rounds, K timed rounds (device time of
+    kvc_update_beacons + kvc_compress on the library's stream), the rooflines
+    of the round's kernels and, for the serving workloads, the end-to-end
+    figure.  Returns (JSON dict, workload, selector)."""
     import numpy as np
     import torch
 
@@ -306,12 +393,15 @@ def run_ours(args, rank, world, dist):
 
     def one_round(seed, timed):
         ev0 = torch.cuda.Event(enable_timing=True)
+        ev_mid = torch.cuda.Event(enable_timing=True)
         ev1 = torch.cuda.Event(enable_timing=True)
         ev0.record(ctx.stream)
-        upd_ms = ctx.update_beacons(timed=timed) if beacon else 0.0
+        if beacon:
+            ctx.update_beacons()
+        ev_mid.record(ctx.stream)
         st = ctx.compress(sel, budgets, seed, stats=timed, **opts)
         ev1.record(ctx.stream)
-        return ev0, ev1, st, upd_ms
+        return ev0, ev_mid, ev1, st
 
     # the first compress brings the cache from its filled length to the budget;
     # from then on every round sees L = K + trigger
@@ -337,51 +427,25 @@ def run_ours(args, rank, world, dist):
         dist.barrier()
     wall = time.perf_counter() - t_wall
     clocks = clock.stop()
-    ms = [a.elapsed_time(b) for a, b, _, _ in rounds]
-    stats = [s for _, _, s, _ in rounds]
-    upd = [u for _, _, _, u in rounds]
+    ms = [a.elapsed_time(c) for a, _, c, _ in rounds]
+    upd = [a.elapsed_time(b) for a, b, _, _ in rounds]
+    stats = [s for _, _, _, s in rounds]
     head_pos = stats[-1]["head_positions"]
     value, total_ms = aggregate(sum(ms), head_pos, args.steps, world, dist, dev)
 
-    # roofline of the dominant kernel
+    # rooflines of the round's kernels; the dominant (longest) one is the line's roofline
     peaks, peak_kind = measured_peaks()
-    variant = [] if args.compaction == "ordered" else [args.compaction]
-    variant += [f"block{args.block}"] if args.block != 1 else []
-    variant += [f"sinks{args.sinks}"] if args.sinks is not None else []
-    traffic_key = "/".join([w.name] + variant)
-    sc_ms = statistics.mean(s["ms_select_compact"] for s in stats)
-    score_ms = statistics.mean(s["ms_score"] for s in stats)
-    moved = statistics.mean(s["moved_rows"] for s in stats)
-    cands = statistics.mean(s["candidates"] for s in stats)
-    rb = w.head_dim * (2 if w.dtype == "bf16" else 4)
-    # select+compact: K and V rows read and written once per moved row, the moved
-    # position entries read and written, every candidate's 4-byte key source read
-    sc_bytes = moved * (4 * rb + 8) + cands * 4
-    if beacon and score_ms > sc_ms:
-        B = w.num_beacons
-        key_bytes = statistics.mean(s["key_bytes_scored"] for s in stats)
-        keys = key_bytes / rb
-        flops = 2.0 * B * w.head_dim * (keys + cands)  # pass 1 over all keys, pass 2 over candidates
-        score_bytes = key_bytes + cands * 4 + (w.segments * B * w.head_dim * (2 if w.dtype == "bf16" else 4))
-        roof = score_roofline(flops, score_bytes, score_ms, peaks, clocks, stats[-1].get("score_kernel", 0) == 2)
-        roof["traffic"] = profiled_traffic(roof["kernel"], w.name, keys)
-    else:
-        roof = {"kernel": "select_compact", "bound": "hbm", "achieved": sc_bytes / (sc_ms / 1e3) / 1e9,
-                "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "traffic": profiled_traffic("select_compact", traffic_key, moved)}
-    roof["frac"] = roof["achieved"] / roof["peak"] if roof.get("peak") else None
-    roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})"
-    roof["algorithmic_bytes_per_launch"] = sc_bytes if roof["kernel"] == "select_compact" else score_bytes
-    if roof["kernel"] != "select_compact":
-        roof["algorithmic_flops_per_launch"] = flops
-    roof["launch_ms"] = sc_ms if roof["kernel"] == "select_compact" else score_ms
+    peaks = dict(peaks, _kind=peak_kind)
+    roofs = round_rooflines(w, sel, stats, upd, peaks, args)
+    dominant = max(roofs, key=lambda k: roofs[k]["launch_ms"])
+    roof = dict(roofs[dominant])
 
     # end to end through the public API, every step: the next trigger window's
     # K/V (and queries) copied H2D from page-locked host memory on a second
     # stream while the round runs, the round, the new lengths read back, then
     # the window appended from device memory once both are done
     e2e = None
-    if not args.no_e2e and refill.window is not None:
+    if with_e2e and not args.no_e2e and refill.window is not None:
         _, k_win, v_win, q_win = refill.window
         k_h = k_win.cpu().pin_memory()
         v_h = v_win.cpu().pin_memory()
@@ -424,7 +488,12 @@ def run_ours(args, rank, world, dist):
                        "memory on a second stream, overlapped with kvc_compress (+kvc_update_beacons); the new "
                        "lengths D2H; the window appended from device memory through kvc_append"}
     ctx.sync()
+    ctx.close()
+    del ctx, refill, gen
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
     launches = sum(s["launches"] for s in stats) + (args.steps if beacon else 0)
+    ragged = len(set(w.length.tolist())) > 1
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -441,10 +510,15 @@ def run_ours(args, rank, world, dist):
                    "head_positions_per_round_per_gpu": head_pos,
                    "parallelism": f"replicas x{world} (no collective on the data path)",
                    "l2": "inputs larger than L2: the cache is tens of GB vs 126 MB L2, and each "
-                         "trigger append between rounds writes >1 GB"},
+                         "refill between rounds writes >1 GB",
+                   **({"layer_slice": f"{w.num_layers} of 36 layers (K+V of all 36 would be ~174 GB); "
+                                      "segments are independent"} if ragged else {})},
         "roofline": roof,
+        "rooflines": roofs,
         "moved_rows_per_round": [int(s["moved_rows"]) for s in stats],
-        "phases_ms": {"select_compact": sc_ms, "score": score_ms, "update": statistics.mean(upd) if beacon else 0.0},
+        "phases_ms": {"update": statistics.mean(upd) if beacon else 0.0,
+                      "score": statistics.mean(s["ms_score"] for s in stats),
+                      "select_compact": statistics.mean(s["ms_select_compact"] for s in stats)},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
@@ -707,6 +781,20 @@ def oracle_pool_rate(args, budget_s: float):
                               f"(one per host core), each ~{budget_s:.0f} s of oracle time")
 
 
+def add_cpu_baselines(out, args, w, sel, single_s: float, pool_s: float, pool: bool):
+    """The oracle on one host core (cpu_baseline) and, unless disabled, on
+    every host core (cpu_baseline_all_cores), on bounded samples of the same
+    workload."""
+    rate, desc, _ = oracle_sample_rate(w, sel, single_s)
+    out["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+    if pool:
+        xa = argparse.Namespace(**vars(args))
+        xa.selector = sel
+        prate, cores, pdesc = oracle_pool_rate(xa, pool_s)
+        out["cpu_baseline_all_cores"] = {"value": prate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                         "sample": pdesc}
+
+
 def run_reference(args, rank, world):
     """The reference arm: the CPU oracle as it stands, on the host cores."""
     if args.phase == "attention":
@@ -724,7 +812,9 @@ def run_reference(args, rank, world):
         return {
             "impl": "reference", "metric": ATTN_METRIC, "value": value, "unit": "head-positions/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": positions / value * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": positions / value * 1e3,
+            "ms_per_step_kind": "extrapolated from the oracle's rate on the sampled units",
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name + "/decode_attention"},
             "cpu_baseline": {"value": value, "unit": "head-positions/s", "cores": 1, "kind": "oracle",
@@ -744,6 +834,9 @@ def run_reference(args, rank, world):
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.head_positions / value * 1e3,
+        "ms_per_step_kind": "extrapolated: one whole round's head-positions divided by the oracle's rate on the "
+                            "sampled segments (a whole round would take this long; each timed step is a bounded "
+                            "sample)",
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": w.name, "selector": sel},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
@@ -779,14 +872,23 @@ def main():
                 print(json.dumps(out), flush=True)
             return
         out, w, sel = run_ours(args, rank, world, dist)
+        if rank == 0 and not args.no_cpu_baseline:
+            add_cpu_baselines(out, args, w, sel, 12.0, 10.0, pool=not args.no_cpu_pool)
+        # the other workloads, fewer rounds each, under extra keys of the same line
+        extras = [x for x in args.extras.split(",") if x and x != args.workload] if args.phase == "round" else []
+        if extras:
+            out["extra_workloads"] = {}
+        for name in extras:
+            xa = argparse.Namespace(**vars(args))
+            xa.workload, xa.selector, xa.requests, xa.layers = name, None, None, None
+            xa.steps, xa.warmup = max(2, args.extra_steps), max(3, min(args.warmup, 3))
+            xo, xw, xsel = run_ours(xa, rank, world, dist, with_e2e=False)
+            if rank == 0 and not args.no_cpu_baseline:
+                add_cpu_baselines(xo, xa, xw, xsel, 6.0, 6.0, pool=not args.no_cpu_pool)
+            for k in ("metric", "unit", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "data", "e2e"):
+                xo.pop(k, None)
+            out["extra_workloads"][name] = xo
         if rank == 0:
-            if not args.no_cpu_baseline:
-                rate, desc, _ = oracle_sample_rate(w, sel, 12.0)
-                out["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
-                if args.cpu_pool:
-                    prate, cores, pdesc = oracle_pool_rate(args, 10.0)
-                    out["cpu_baseline_all_cores"] = {"value": prate, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                                     "sample": pdesc}
             print(json.dumps(out), flush=True)
     finally:
         if dist:

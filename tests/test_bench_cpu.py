@@ -1,5 +1,6 @@
-"""bench.py's roofline bookkeeping on the CPU: the score kernel's bound and
-peak choice, and the traffic lookup gated by the kernel sources' hash."""
+"""bench.py's roofline bookkeeping on the CPU: the score kernel's bound, peak
+and flop count, the update kernel's bytes, and the traffic lookup gated by the
+kernel sources' hash."""
 import json
 import os
 
@@ -11,31 +12,49 @@ PEAKS = {"hbm_gbs": 6529.4, "bf16_tflops": 1674.6, "bf16_tflops_sustained": 1388
 
 
 def test_score_roofline_hbm_below_ridge():
-    # 64 flop per byte is under both ridges (256 burst, 213 sustained)
-    r = bench.score_roofline(64e12, 1e12, 1000.0, PEAKS, {"reasons": []}, True)
+    # 64 flop per byte is under the burst ridge (1674.6 TFLOP/s / 6529.4 GB/s = 256.5)
+    r = bench.score_roofline(64e12, 1e12, 1000.0, PEAKS, True)
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert r["achieved"] == pytest.approx(1000.0) and r["peak"] == PEAKS["hbm_gbs"]
     assert r["flop_per_byte"] == pytest.approx(64.0)
+    assert r["tensor_frac"] == pytest.approx(64.0 / 1674.6)
 
 
-@pytest.mark.parametrize("reasons,peak,kind", [([], 1674.6, "burst"), (["sw_power_cap"], 1388.6, "sustained")])
-def test_score_roofline_tensor_above_ridge(reasons, peak, kind):
-    r = bench.score_roofline(500e12, 1e12, 1000.0, PEAKS, {"reasons": reasons}, True)
+def test_score_roofline_tensor_above_ridge_uses_the_burst_peak():
+    r = bench.score_roofline(500e12, 1e12, 1000.0, PEAKS, True)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
-    assert r["peak"] == peak and r["peak_kind"] == kind
+    assert r["peak"] == 1674.6 and r["peak_kind"] == "burst"
     assert r["achieved"] == pytest.approx(500.0)
+    assert r["hbm_frac"] == pytest.approx(1000.0 / 6529.4)
 
 
-def test_score_roofline_ridge_follows_the_peak():
-    # 230 flop per byte: tensor-bound against the sustained ridge (213), HBM-bound against the burst one (256)
-    assert bench.score_roofline(230e12, 1e12, 1.0, PEAKS, {"reasons": ["sw_power_cap"]}, True)["bound"] == "tensor"
-    assert bench.score_roofline(230e12, 1e12, 1.0, PEAKS, {"reasons": []}, True)["bound"] == "hbm"
+def test_score_roofline_ridge():
+    assert bench.score_roofline(257e12, 1e12, 1.0, PEAKS, True)["bound"] == "tensor"
+    assert bench.score_roofline(256e12, 1e12, 1.0, PEAKS, True)["bound"] == "hbm"
+
+
+def test_score_roofline_counts_the_recompute_apart():
+    # the method's work is one product per (beacon, key) pair; pass 2's recompute is reported, not counted
+    r = bench.score_roofline(300e12, 1e12, 1000.0, PEAKS, True, recompute_flops=290e12)
+    assert r["achieved"] == pytest.approx(300.0)
+    assert r["executed_tflops"] == pytest.approx(590.0)
+    assert r["algorithmic_flops_per_launch"] == 300e12 and r["recompute_flops_per_launch"] == 290e12
 
 
 def test_score_roofline_simt():
-    r = bench.score_roofline(74.4e12, 1e12, 1000.0, PEAKS, None, False)
+    r = bench.score_roofline(74.4e12, 1e12, 1000.0, PEAKS, False)
     assert r["bound"] == "alu" and r["kernel"] == "beacon_score_simt"
     assert r["peak"] == pytest.approx(148 * 128 * 2 * 1965e6 / 1e12)
+
+
+def test_update_roofline_bytes():
+    import types
+    w = types.SimpleNamespace(dtype="bf16", num_beacons=64, head_dim=128, query_window=64, G=4, segments=36864)
+    r = bench.update_roofline(w, 2.0, PEAKS, True)
+    per_seg = 64 * 4 * 128 * 2 + 64 * 128 * 10 + 64 * 12
+    assert r["algorithmic_bytes_per_launch"] == 36864 * per_seg
+    assert r["achieved"] == pytest.approx(36864 * per_seg / 2e-3 / 1e9)
+    assert r["bound"] == "hbm" and r["kernel"] == "beacon_update_tc"
 
 
 def test_traffic_lookup_gated_by_source_hash(tmp_path, monkeypatch):
