@@ -36,9 +36,13 @@
  *  - Ordering: every call is enqueued on the context's CUDA stream and is
  *    asynchronous unless stated.  Host arrays passed in are consumed before
  *    the call returns.  A context is not thread-safe.
- *  - Device-detected errors (KVC_ERR_NAN, KVC_ERR_DEVICE_CHECK) are latched
+ *  - Device-detected errors (KVC_ERR_NAN, KVC_ERR_DEVICE_TIMEOUT) are latched
  *    in a device status word and reported by the next synchronising call
- *    (kvc_sync, or a call given a stats pointer).
+ *    (kvc_sync, or a call given a stats pointer).  Page ids, slots and
+ *    lengths reach the kernels only from the library's own bookkeeping
+ *    (kvc_append allocates the pages; kvc_compress frees them), which the
+ *    host validates, so the kernels do not range-check them; a caller that
+ *    writes into the state through kvc_gather_view takes that on itself.
  *
  * Data layout (all row-major, C order):
  *   k_pool, v_pool  [num_layers][num_pages][num_kv_heads][16][head_dim] dtype
@@ -72,8 +76,9 @@ typedef enum {
   KVC_ERR_STATE = 3,          /* call not valid in the current state */
   KVC_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed */
   KVC_ERR_NAN = 5,            /* a NaN reached a beacon distance or score */
-  KVC_ERR_DEVICE_CHECK = 6,   /* a kernel found an index out of range */
-  KVC_ERR_DEVICE_TIMEOUT = 7, /* reserved: a bounded device wait ran out */
+  KVC_ERR_DEVICE_CHECK = 6,   /* reserved, never returned by this build: the value is kept for a
+                                 build whose kernels range-check page ids and slots */
+  KVC_ERR_DEVICE_TIMEOUT = 7, /* a bounded device wait ran out (see kvc_check_wait_timeout) */
   KVC_ERR_UNSUPPORTED = 8     /* valid request this build does not support */
 } kvc_status;
 
@@ -346,7 +351,12 @@ const char *kvc_last_error(const kvc_ctx *ctx);
  *               is left untouched.
  *   cuda_stream: cudaStream_t on the inputs' device (NULL = legacy stream).
  * The scores and the selection are those of kvc_compress(KVC_SEL_BEACON)
- * for the same keys and beacons.  Scratch: the scores pass between the two
+ * for the same keys and beacons.  NaN: this call does not synchronise and
+ * reports no KVC_ERR_NAN; a NaN score (one NaN key or beacon makes every
+ * score of its segment NaN) ranks below every other score, ties among NaN
+ * scores keep the lowest slots, and scores_out shows the NaN.  The kernels
+ * run on the keys' device; the calling thread's current device is the same
+ * after the call as before it.  Scratch: the scores pass between the two
  * kernels through a fixed array of 1,048,576 floats (4 MiB) in the library's
  * device memory, held on every GPU that loads the library until the process
  * exits; S*(L-P) above 1,048,576 is rejected with KVC_ERR_INVALID_ARG.  No
