@@ -15,6 +15,7 @@
 // its order are the same, so the results match kvc_compress(KVC_SEL_BEACON).
 #include <cuda_bf16.h>
 
+#include <memory>
 #include <mutex>
 #include <string>
 
@@ -59,6 +60,33 @@ __device__ __forceinline__ float na_load(const uint8_t *base, int64_t idx) {
     return reinterpret_cast<const float *>(base)[idx];
 }
 
+// Elements of one 16-byte chunk: 8 bf16 or 4 fp32.
+template <int DT>
+struct NaChunk {
+  static constexpr int kElems = DT == KVC_BF16 ? 8 : 4;
+};
+
+// Loads the 16-byte chunk that starts at element idx (16-byte aligned) and
+// widens it to fp32.
+template <int DT>
+__device__ __forceinline__ void na_load_chunk(const uint8_t *base, int64_t idx, float *out) {
+  if (DT == KVC_BF16) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(base + idx * 2));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      out[2 * i] = __uint_as_float(w[i] << 16);
+      out[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  } else {
+    const float4 f = __ldg(reinterpret_cast<const float4 *>(base + idx * 4));
+    out[0] = f.x;
+    out[1] = f.y;
+    out[2] = f.z;
+    out[3] = f.w;
+  }
+}
+
 constexpr int kNT = 256;
 constexpr int kTK = 32;
 constexpr int kNG = kNT / kTK;
@@ -73,16 +101,49 @@ __global__ void __launch_bounds__(kNT)
   float *zs = ks + kTK * (D + 1);
   float *lse = zs + B * (kTK + 1);
   float *red = lse + B;
+  __shared__ int seg_nan;  // a beacon's log-sum-exp is NaN: every score of the segment is NaN
   const int tid = threadIdx.x, s = blockIdx.x;
   const int N = L - P;
   const float inv_sqrt_d = 1.0f / sqrtf((float)D);
-  for (int e = tid; e < B * D; e += kNT) cs[e] = na_load<DT>(beacons, (int64_t)s * B * D + e);
+  if (tid == 0) seg_nan = 0;
+  // 16-byte loads when both inputs start on a 16-byte boundary (a row is
+  // D * sizeof(dtype) bytes, a multiple of 16, so every row chunk is then
+  // aligned too); element loads otherwise.  Same values either way.
+  constexpr int CE = NaChunk<DT>::kElems;
+  constexpr int CPR = D / CE;  // chunks per row
+  const bool vec = (((uintptr_t)keys | (uintptr_t)beacons) & 15) == 0;
+  if (vec) {
+    for (int c = tid; c < B * CPR; c += kNT) {
+      float v[CE];
+      na_load_chunk<DT>(beacons, (int64_t)s * B * D + (int64_t)c * CE, v);
+#pragma unroll
+      for (int i = 0; i < CE; ++i) cs[c * CE + i] = v[i];
+    }
+  } else {
+    for (int e = tid; e < B * D; e += kNT) cs[e] = na_load<DT>(beacons, (int64_t)s * B * D + e);
+  }
   const int jj = tid % kTK, bg = tid / kTK;
   auto load_tile = [&](int j0) {
-    for (int e = tid; e < kTK * D; e += kNT) {
-      const int t = e / D, k = e - t * D;
-      const int j = j0 + t;
-      ks[t * (D + 1) + k] = j < L ? na_load<DT>(keys, ((int64_t)s * L + j) * D + k) : 0.f;
+    if (vec) {
+      for (int c = tid; c < kTK * CPR; c += kNT) {
+        const int t = c / CPR, k = (c - t * CPR) * CE;
+        const int j = j0 + t;
+        float v[CE];
+        if (j < L) {
+          na_load_chunk<DT>(keys, ((int64_t)s * L + j) * D + k, v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < CE; ++i) v[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < CE; ++i) ks[t * (D + 1) + k + i] = v[i];
+      }
+    } else {
+      for (int e = tid; e < kTK * D; e += kNT) {
+        const int t = e / D, k = e - t * D;
+        const int j = j0 + t;
+        ks[t * (D + 1) + k] = j < L ? na_load<DT>(keys, ((int64_t)s * L + j) * D + k) : 0.f;
+      }
     }
   };
   auto dots = [&]() {
@@ -115,7 +176,11 @@ __global__ void __launch_bounds__(kNT)
       for (int t = 0; t < nv; ++t) run_s += expf(z[t] - run_m);
     }
   }
-  if (tid < B) lse[tid] = run_m + logf(run_s);
+  if (tid < B) {
+    const float v = run_m + logf(run_s);
+    lse[tid] = v;
+    if (v != v) seg_nan = 1;  // a NaN key or beacon (fmaxf below would drop it)
+  }
 #pragma unroll 1
   for (int j0 = P; j0 < L; j0 += kTK) {
     __syncthreads();
@@ -130,13 +195,20 @@ __global__ void __launch_bounds__(kNT)
     if (tid < kTK && j0 + tid < L) {
       float m = red[tid];
       for (int g = 1; g < kNG; ++g) m = fmaxf(m, red[g * kTK + tid]);
-      scratch[(int64_t)s * N + (j0 + tid - P)] = expf(m);
+      scratch[(int64_t)s * N + (j0 + tid - P)] = seg_nan ? __int_as_float(0x7fffffff) : expf(m);
     }
   }
 }
 
+// Order-preserving map of a score to an unsigned key.  A NaN score (one NaN
+// key or beacon makes every score of its segment NaN) maps to 0, below every
+// other score, so NaN candidates are the first to go and ties among them keep
+// the lowest slots.  This call does not
+// synchronise, so unlike kvc_compress it reports no KVC_ERR_NAN; callers that
+// need to detect NaN inputs read scores_out.
 __device__ __forceinline__ uint32_t na_order_key(float f) {
   const uint32_t u = __float_as_uint(f);
+  if (f != f) return 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
@@ -287,8 +359,20 @@ extern "C" kvc_status kvc_beacon_select_noalloc(const void *keys, const void *be
     set_thread_error(std::string("kvc_beacon_select_noalloc: ") + what + ": " + cudaGetErrorString(e));
     return KVC_ERR_CUDA;
   };
-  cudaError_t e = cudaSetDevice(dev);
-  if (e != cudaSuccess) return cuda_err(e, "cudaSetDevice");
+  // The launches go to the keys' device; the caller's current device is put
+  // back on every return path.
+  int prev_dev = -1;
+  cudaError_t e = cudaGetDevice(&prev_dev);
+  if (e != cudaSuccess) return cuda_err(e, "cudaGetDevice");
+  struct RestoreDevice {
+    int dev;
+    ~RestoreDevice() { cudaSetDevice(dev); }
+  };
+  std::unique_ptr<RestoreDevice> restore;
+  if (prev_dev != dev) {
+    if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_err(e, "cudaSetDevice");
+    restore.reset(new RestoreDevice{prev_dev});
+  }
   float *scratch = nullptr;
   if ((e = scratch_address(dev, &scratch)) != cudaSuccess) return cuda_err(e, "cudaGetSymbolAddress");
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);

@@ -16,7 +16,9 @@ these synthetic inputs stand in for them:
 * decode queries from a mixture of von Mises-Fisher distributions on the unit
   sphere (per (layer, KV head) a set of component means uniform on the
   sphere; each (request, step, query head) picks a component uniformly and
-  draws with concentration kappa = 20, Wood's 1994 rejection sampler);
+  draws with concentration kappa = 20, Wood's 1994 rejection sampler), or,
+  for the "sharp" test variants, the same directions scaled to norm sqrt(d)
+  so that beacon scores spread far from the uniform 1/L;
 * ragged lengths L_r ~ U{4096..32768} and prompts P_r ~ U{128..1536}.
 """
 from __future__ import annotations
@@ -44,6 +46,7 @@ class Workload:
     query_window: int = 0
     n_components: int = 0
     kappa: float = 20.0
+    query_norm: float = 1.0  # queries lie on the sphere of this radius (sqrt(d) spreads the scores)
     outlier_channels: int = 4
     outlier_scale: float = 8.0
     trigger: int = 64       # tokens appended between rounds at steady state
@@ -194,10 +197,12 @@ class Generator:
             todo = todo[~ok]
         return out
 
-    def queries(self, n_req: int, T: int, norm: float = 1.0):
-        """Decode queries [n_req, layers, T, Hq, d] from the vMF mixture."""
+    def queries(self, n_req: int, T: int, norm: float | None = None):
+        """Decode queries [n_req, layers, T, Hq, d] from the vMF mixture, scaled to
+        the workload's query norm unless ``norm`` is given."""
         import torch
         w = self.w
+        norm = w.query_norm if norm is None else norm
         Ly, Hq, d = w.num_layers, w.num_q_heads or w.num_kv_heads, w.head_dim
         out = torch.empty((n_req, Ly, T, Hq, d), dtype=self.dtype, device=self.device)
         per_req = Ly * T * Hq * d * 8 * 4  # float64 temporaries

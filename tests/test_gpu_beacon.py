@@ -4,8 +4,15 @@ Staged parity: the oracle's beacon update is compared assignment by
 assignment (exact, or a counted near-tie), then recomputed from the GPU's
 assignments (fp32 vs double running means); the oracle's scores are computed
 from the GPU's scoring copy of the beacons and the pre-round keys, then
-compared within |g - o| <= 1e-5 + 1e-3|o|; the kept set must match the
-oracle's except within 1e-4 of the threshold, with equal counts."""
+compared within |g - o| <= 1e-5 + 1e-3|o| and within the strict relative
+gate |g - o| <= 1e-9 + 1e-4|o|; the kept set must match the oracle's except
+within 1e-4*tau of the threshold tau, with equal counts.
+
+The "sharp" cases scale the decode queries to norm sqrt(d): beacons are then
+long enough that the softmax over the keys is far from uniform, and scores
+spread over several orders of magnitude instead of sitting near 1/L."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -75,7 +82,9 @@ def run_beacon(w, sample=None, score_impl=None, sinks=None, compaction="ordered"
     # the scoring copy is the fp32 beacon rounded to the cache dtype (torch's RNE cast)
     assert torch.equal(st["beacons_scoring"], st["beacons"].to(ctx.dtype))
     segs = [(r, l, h) for r in range(R) for l in range(Ly) for h in range(H)]
-    if sample is not None:
+    if isinstance(sample, list):
+        segs = list(sample)  # explicit (request, layer, head) segments
+    elif sample is not None:
         segs = [segs[i] for i in np.random.default_rng(0).choice(len(segs), sample, replace=False)]
     near_ties = 0
     for (r, l, h) in segs:
@@ -178,12 +187,20 @@ def test_beacon_serving_full_size_sampled():
     print(out)
 
 
-@pytest.mark.parametrize("c", [2, 16])
+@pytest.mark.parametrize("c", [2, 4, 8, 16])
 def test_ragged_beacon_sampled(c):
-    """Ragged lengths 4096..32768 (the ragged sweep's first 4 requests, 2 layers) at 2x and 16x compression,
-    including prompts over budget at 16x: sampled segments."""
+    """Ragged lengths 4096..32768 (the ragged sweep's first 4 requests, 2 layers) at 2x, 4x, 8x and 16x
+    compression, including prompts close to and over the budget: sampled segments."""
     w = wl.scaled(wl.ragged(c), num_requests=4, num_layers=2)
     out = run_beacon(w, sample=12)
+    print(c, out)
+
+
+@pytest.mark.parametrize("c", [4, 8])
+def test_ragged_cluster_trigger_sampled(c):
+    """The cluster-trigger selector on a ragged slice (first 4 requests, 2 layers) at 4x and 8x."""
+    w = wl.scaled(wl.ragged(c), num_requests=4, num_layers=2)
+    out = run_beacon(w, sample=12, selector="beacon_trigger")
     print(c, out)
 
 
@@ -191,6 +208,40 @@ def test_long_trace_sampled():
     w = wl.scaled(wl.long_trace(), num_requests=2, num_layers=4)
     out = run_beacon(w, sample=3)
     print(out)
+
+
+def test_long_trace_every_request():
+    """All 8 requests of the long trace (two layers of 32768 keys each, 256 beacons): one sampled segment of
+    every request, on alternating layers and heads."""
+    w = wl.scaled(wl.long_trace(), num_layers=2)
+    segs = [(r, r % 2, (3 * r) % 8) for r in range(8)]
+    out = run_beacon(w, sample=segs)
+    print(out)
+
+
+def _sharp(w):
+    return wl.scaled(w, query_norm=math.sqrt(w.head_dim))
+
+
+@pytest.mark.parametrize("selector", ["beacon", "beacon_trigger"])
+@pytest.mark.parametrize("impl", [1, 2], ids=["simt", "tcgen05"])
+def test_sharp_beacon_serving(impl, selector):
+    """Queries of norm sqrt(d) at the beacon-serving shape (3 requests, 2 layers, every segment), both score
+    kernels and both beacon selectors, under the strict gate."""
+    out = run_beacon(_sharp(wl.beacon_serving(R=3, layers=2)), score_impl=impl, selector=selector)
+    print(impl, selector, out)
+    assert out["max_rel_score_err"] < 1e-4
+
+
+@pytest.mark.parametrize("selector", ["beacon", "beacon_trigger"])
+@pytest.mark.parametrize("impl", [1, 2], ids=["simt", "tcgen05"])
+def test_sharp_long_trace(impl, selector):
+    """Queries of norm sqrt(d) at the long-trace shape (32768 keys, 256 beacons; 2 requests, 2 layers,
+    4 sampled segments), both score kernels and both beacon selectors, under the strict gate."""
+    w = _sharp(wl.scaled(wl.long_trace(), num_requests=2, num_layers=2))
+    out = run_beacon(w, sample=[(0, 0, 1), (0, 1, 6), (1, 0, 4), (1, 1, 3)], score_impl=impl, selector=selector)
+    print(impl, selector, out)
+    assert out["max_rel_score_err"] < 1e-4
 
 
 @pytest.mark.parametrize("sinks,compaction", [(4, "ordered"), (None, "hole_fill"), (0, "hole_fill")])
