@@ -148,9 +148,11 @@ def test_serving_full_size():
     run_rounds(w, "random", rounds=2, seed=w.philox_seed, kv_layers=[0, 35], check_scores_n=2000)
 
 
-def test_ragged_sweep_slice():
-    """Ragged lengths 4096..32768 with prompts 128..1536 at 2x and 16x compression
-    (12-layer slice), random and shared selectors: every position map."""
-    for c, sel in [(2, "random"), (16, "random_shared")]:
-        w = wl.scaled(wl.ragged(c), num_layers=12, num_beacons=0, query_window=0, num_q_heads=8)
-        run_rounds(w, sel, rounds=1, seed=w.philox_seed, kv_layers=[5], check_scores_n=500)
+@pytest.mark.parametrize("c,sel", [(2, "random"), (4, "random"), (4, "random_shared"), (8, "random"),
+                                   (8, "random_shared"), (16, "random_shared")])
+def test_ragged_sweep_slice(c, sel):
+    """Ragged lengths 4096..32768 with prompts 128..1536 at 2x, 4x, 8x and 16x compression (12-layer slice; at
+    4x and 8x some prompts come close to or over the budget), random and shared selectors: every position map,
+    the K/V bytes of one layer and a sample of the 32-bit draws."""
+    w = wl.scaled(wl.ragged(c), num_layers=12, num_beacons=0, query_window=0, num_q_heads=8)
+    run_rounds(w, sel, rounds=1, seed=w.philox_seed, kv_layers=[5], check_scores_n=500)
