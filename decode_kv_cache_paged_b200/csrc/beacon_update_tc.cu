@@ -343,6 +343,494 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Pipelined form for up to 128 beacons.  One persistent CTA per SM walks its
+// segments; the work is split by role so that the point loads, the beacon
+// preparation, the products, the argmins and the running means of
+// neighbouring tiles and segments overlap instead of running as one serial
+// chain per segment:
+//   warp 0      TMEM allocation and the MMA issuer (one lane); within a
+//               segment the assignment product of tile g+1 is issued before
+//               the sums of tile g, and a segment's last sums before the next
+//               segment's first assignment;
+//   warps 1-4   point warps: one point per thread.  Each thread copies its
+//               point of the tile D ahead with cp.async into one of NXS
+//               stages (128-byte-swizzled K-major layout; rows past the
+//               segment's points zero-filled), then takes the argmin over its
+//               TMEM lane of the assignment product, writes its one-hot entry
+//               and counts it;
+//   warps 5-8   preparation: the next segment's beacons as bf16 hi/lo terms
+//               (swizzled, the B operand of the assignment) and their fp32
+//               squared norms;
+//   warps 9-12  running mean: one dimension per thread, over every beacon.
+// The sums are D[dim][beacon] = X^T OH, with the point tile read as an
+// MN-major A operand (dimensions on M, its 64-dimension blocks 16 KB apart)
+// and the one-hot tile OH [beacon rows x point columns] as a K-major B
+// operand: a segment's sums take B TMEM columns, and the running mean reads
+// and writes each beacon row with one coalesced access per warp.
+// TMEM columns: two assignment buffers of BM, then two sums buffers of BM
+// (sums of neighbouring segments alternate).  The counts of three segments
+// rotate in shared memory so that the preparation never waits for a mean.
+// Every wait is bounded.
+constexpr int kPipeWarps = 13;
+constexpr int kPipeThreads = 32 * kPipeWarps;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Every lane of the warp waits (bounded); the warp takes one decision.
+__device__ __forceinline__ bool lanes_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                           int32_t *status) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, status);
+  return __all_sync(0xffffffffu, ok);
+}
+
+struct PipeSeg {
+  int r, l, h, n_pts, T, init, ring_start;
+  int64_t seg;
+};
+__device__ __forceinline__ PipeSeg pipe_seg(const BeaconUpdateParams &p, int s) {
+  PipeSeg g;
+  g.h = s % p.hkv;
+  g.l = (s / p.hkv) % p.layers;
+  const UpdateDesc ud = p.descs[s / (p.hkv * p.layers)];
+  g.r = ud.req;
+  g.n_pts = ud.n_steps * p.G;
+  g.T = (g.n_pts + 127) / 128;
+  g.init = ud.init;
+  g.ring_start = ud.ring_start;
+  g.seg = ((int64_t)g.r * p.layers + g.l) * p.hkv + g.h;
+  return g;
+}
+// Element offset in the query ring of point pt of the segment (step pt / G,
+// query head h*G + pt % G of the step's ring slot).
+__device__ __forceinline__ int64_t pipe_point(const BeaconUpdateParams &p, const PipeSeg &g, int pt) {
+  const int step = pt / p.G, gq = pt - step * p.G;
+  int slot = g.ring_start + step;
+  if (slot >= p.W) slot -= p.W;
+  return ((((int64_t)g.r * p.layers + g.l) * p.W + slot) * p.hq + (g.h * p.G + gq)) * 128;
+}
+
+template <int BM, int NXS, int NCB, int DA>
+__global__ void __launch_bounds__(kPipeThreads, 1)
+    beacon_update_pipe_kernel(BeaconUpdateParams p, int n_segs) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_align<1024>(smem_raw);
+  constexpr int D = 128;
+  constexpr uint32_t kXBytes = 32768;    // 128 points x 128 bf16
+  constexpr uint32_t kCBytes = BM * 256;  // one term of one beacon buffer: [2 K-blocks][B rows][128 B]
+  constexpr uint32_t kOHBytes = BM * 256; // one one-hot tile: [2 point blocks][B rows][128 B]
+  const int B = p.B;
+  uint8_t *xs = smem;
+  uint8_t *chi = xs + NXS * kXBytes;
+  uint8_t *clo = chi + NCB * kCBytes;
+  uint8_t *oh = clo + NCB * kCBytes;
+  float *cn = reinterpret_cast<float *>(oh + 2 * kOHBytes);     // [NCB][BM] squared norms
+  float *cpart = cn + NCB * BM;                                   // [2][4][BM] per-warp partial norms
+  int32_t *cnt = reinterpret_cast<int32_t *>(cpart + 8 * BM);    // [3][BM] this update's counts
+  int32_t *nold = cnt + 3 * BM;                                   // [2][BM] counts before the update
+  uint64_t *bars = reinterpret_cast<uint64_t *>(nold + 2 * BM);
+  uint64_t *x_full = bars, *x_empty = x_full + NXS;
+  uint64_t *prep_full = x_empty + NXS, *prep_empty = prep_full + NCB;
+  uint64_t *cnt_full = prep_empty + NCB, *cnt_empty = cnt_full + 3;
+  uint64_t *acc_full = cnt_empty + 3, *acc_empty = acc_full + 2;
+  uint64_t *oh_full = acc_empty + 2, *oh_empty = oh_full + 2;
+  uint64_t *sum_full = oh_empty + 2, *sum_empty = sum_full + 2;
+  uint64_t *prep_sync = sum_empty + 2, *mean_sync = prep_sync + 1, *mma_done = mean_sync + 1;
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(mma_done + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if (tid == 0) {
+    for (int i = 0; i < NXS; ++i) {
+      mbar_init(&x_full[i], 128);  // the point threads' copies
+      mbar_init(&x_empty[i], 1);
+    }
+    for (int i = 0; i < NCB; ++i) {
+      mbar_init(&prep_full[i], 128);
+      mbar_init(&prep_empty[i], 1 + 128);  // MMA commit, point warps
+    }
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&cnt_full[i], 128);   // point warps: the segment's counts are complete
+      mbar_init(&cnt_empty[i], 128);  // mean warps: read and zeroed again
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+      mbar_init(&oh_full[i], 128);
+      mbar_init(&oh_empty[i], 1);
+      mbar_init(&sum_full[i], 1);
+      mbar_init(&sum_empty[i], 128);
+    }
+    mbar_init(prep_sync, 128);
+    mbar_init(mean_sync, 128);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // the one-hot tiles start at zero (each point clears its own entry later),
+  // and so do the count buffers (the mean warps zero each after reading it)
+  for (int i = tid; i < (int)(2 * kOHBytes / 16); i += kPipeThreads)
+    reinterpret_cast<uint4 *>(oh)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = tid; i < 3 * BM; i += kPipeThreads) cnt[i] = 0;
+  fence_proxy_async();
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                 "r"(4 * BM));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t tmem_base = *tslot;
+  const __nv_bfloat16 *ring = reinterpret_cast<const __nv_bfloat16 *>(p.qring);
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_asg = idesc_bf16_f32(128, B);
+      const uint32_t idesc_sum = idesc_bf16_f32(128, B) | (1u << 15);  // A (the point tile) MN-major
+      bool ok = true;
+      auto assign = [&](uint32_t gi, int si, int t, int T) {
+        const int cb = si % NCB;
+        if (t == 0) ok = ok && mbar_wait(&prep_full[cb], (si / NCB) & 1, abort_flag, p.status);
+        ok = ok && mbar_wait(&x_full[gi % NXS], (gi / NXS) & 1, abort_flag, p.status) &&
+             mbar_wait(&acc_empty[gi & 1], ((gi >> 1) & 1) ^ 1, abort_flag, p.status);
+        if (!ok) return;
+        tmem_fence_after();
+        const uint32_t xa = smem_u32(xs + (gi % NXS) * kXBytes);
+        const uint32_t ha = smem_u32(chi + cb * kCBytes), la = smem_u32(clo + cb * kCBytes);
+        for (int term = 0; term < 2; ++term)
+          for (int kb = 0; kb < 2; ++kb)
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t a = sw128_desc(xa + kb * 16384 + ks * 32);
+              const uint64_t bd = sw128_desc((term ? la : ha) + kb * B * 128 + ks * 32);
+              umma(tmem_base + (gi & 1) * BM, a, bd, idesc_asg, (term | kb | ks) != 0);
+            }
+        umma_commit(&acc_full[gi & 1]);
+        if (t == T - 1) umma_commit(&prep_empty[cb]);  // the beacon terms have been read
+      };
+      auto sums = [&](uint32_t gi, int si, int t, int T) {
+        const int sb = si & 1;
+        ok = ok && mbar_wait(&oh_full[gi & 1], (gi >> 1) & 1, abort_flag, p.status);
+        if (t == 0) ok = ok && mbar_wait(&sum_empty[sb], ((si >> 1) & 1) ^ 1, abort_flag, p.status);
+        if (!ok) return;
+        tmem_fence_after();
+        const uint32_t xa = smem_u32(xs + (gi % NXS) * kXBytes), oa = smem_u32(oh + (gi & 1) * kOHBytes);
+        for (int ks = 0; ks < 8; ++ks) {
+          // X^T: 16 points from point group ks, 64-dimension blocks 16 KB apart (LBO), 8-point groups 1 KB
+          // apart (SBO)
+          uint64_t a = sw128_desc(xa + ks * 2048);
+          a = (a & ~(uint64_t)(0x3FFFull << 16)) | ((uint64_t)(16384 >> 4) << 16);
+          const uint64_t bd = sw128_desc(oa + (ks >> 2) * B * 128 + (ks & 3) * 32);
+          umma(tmem_base + 2 * BM + sb * BM, a, bd, idesc_sum, (t > 0 || ks > 0) ? 1u : 0u);
+        }
+        umma_commit(&x_empty[gi % NXS]);
+        umma_commit(&oh_empty[gi & 1]);
+        if (t == T - 1) umma_commit(&sum_full[sb]);
+      };
+      // tile stream; the assignment runs one tile ahead of the sums
+      uint32_t gi = 0;
+      int si = 0;
+      bool have_prev = false;
+      uint32_t pg = 0;
+      int ps = 0, pt = 0, pT = 0;
+      // within a segment; at a segment boundary the last sums go first, so
+      // that the running mean of a segment never waits for the next
+      // segment's beacon preparation
+      for (int s = blockIdx.x; s < n_segs && ok; s += gridDim.x, ++si) {
+        const PipeSeg g = pipe_seg(p, s);
+        for (int t = 0; t < g.T && ok; ++t, ++gi) {
+          if (have_prev && t == 0) sums(pg, ps, pt, pT);
+          assign(gi, si, t, g.T);
+          if (have_prev && t > 0) sums(pg, ps, pt, pT);
+          have_prev = true;
+          pg = gi;
+          ps = si;
+          pt = t;
+          pT = g.T;
+        }
+      }
+      if (have_prev && ok) sums(pg, ps, pt, pT);
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, abort_flag, p.status, false);
+    }
+    __syncwarp();
+  } else if (warp < 5) {
+    // --------------------------------------------------------- point warps
+    const int q = warp & 3, row = q * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    const int NP = p.W * p.G;
+    uint32_t gi = 0;
+    int si = 0;
+    bool ok = true, nan = false;
+    uint32_t last_off0 = 0xffffffffu, last_off1 = 0xffffffffu;  // this point's entry in each one-hot tile
+    // load stream, DA tiles ahead of the argmins: this thread's point row of
+    // tile gl goes to stage gl % NXS
+    int ls = blockIdx.x, lt = 0;
+    bool lvalid = ls < n_segs;
+    PipeSeg lg = pipe_seg(p, lvalid ? ls : 0);
+    uint32_t gl = 0;
+    auto issue = [&]() -> bool {
+      const int st = gl % NXS;
+      if (!lanes_wait(&x_empty[st], ((gl / NXS) & 1) ^ 1, abort_flag, p.status)) return false;
+      uint8_t *dst = xs + st * kXBytes + row * 128;
+      const int pt = lt * 128 + row;
+      const bool valid = pt < lg.n_pts;
+      const __nv_bfloat16 *src = valid ? ring + pipe_point(p, lg, pt) : ring;
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        cp_async16(smem_u32(dst + (c >> 3) * 16384 + (((c & 7) ^ (row & 7)) << 4)), valid ? src + c * 8 : ring,
+                   valid ? 16u : 0u);
+      cp_async_commit();
+      ++gl;
+      if (++lt == lg.T) {
+        lt = 0;
+        ls += gridDim.x;
+        lvalid = ls < n_segs;
+        if (lvalid) lg = pipe_seg(p, ls);
+      }
+      return true;
+    };
+    for (int d = 0; d < DA && lvalid && ok; ++d) ok = issue();
+    // tile 0 is handed to the MMA here, tile g+1 at the start of iteration g,
+    // so that the assignment of tile g+1 runs during the argmin of tile g
+    uint32_t gs = 0;  // tiles handed to the MMA so far
+    auto hand = [&]() {
+      // tile gs has landed once at most gl - gs - 1 later groups are pending
+      if (DA >= 2 && gl - gs >= 2) cp_async_wait<1>();
+      else cp_async_wait<0>();
+      fence_proxy_async();
+      mbar_arrive(&x_full[gs % NXS]);
+      ++gs;
+    };
+    if (ok && gl > 0) hand();
+    for (int s = blockIdx.x; s < n_segs && ok; s += gridDim.x, ++si) {
+      const PipeSeg g = pipe_seg(p, s);
+      const int cb = si % NCB, kb3 = si % 3;
+      ok = lanes_wait(&prep_full[cb], (si / NCB) & 1, abort_flag, p.status) &&
+           lanes_wait(&cnt_empty[kb3], ((si / 3) & 1) ^ 1, abort_flag, p.status);
+      if (!ok) break;
+      const float *cnb = cn + cb * BM;
+      int32_t *cntb = cnt + kb3 * BM;
+      for (int t = 0; t < g.T; ++t, ++gi) {
+        if (gs < gl) hand();  // tile gi + 1
+        if (lvalid) ok = issue();
+        if (!ok) break;
+        const int ab = gi & 1;
+        ok = lanes_wait(&acc_full[ab], (gi >> 1) & 1, abort_flag, p.status);
+        if (!ok) break;
+        tmem_fence_after();
+        float best = __int_as_float(0x7f800000);
+        int besti = 0;
+        for (int c0 = 0; c0 < B; c0 += 32) {
+          float v[32];
+          tmem_ld32(tmem_base + lane_addr + ab * BM + c0, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float dist = fmaf(-2.f, v[i], cnb[c0 + i]);
+            nan |= (dist != dist);
+            if (dist < best) {
+              best = dist;
+              besti = c0 + i;
+            }
+          }
+        }
+        tmem_fence_before();
+        mbar_arrive(&acc_empty[ab]);
+        const int pt = t * 128 + row;
+        const bool valid = pt < g.n_pts;
+        if (valid) {
+          if (p.assign_out) p.assign_out[g.seg * (int64_t)NP + pt] = besti;
+          atomicAdd(&cntb[besti], 1);
+        }
+        ok = lanes_wait(&oh_empty[ab], ((gi >> 1) & 1) ^ 1, abort_flag, p.status);
+        if (!ok) break;
+        uint8_t *ohb = oh + ab * kOHBytes;
+        const uint32_t prev = ab ? last_off1 : last_off0;
+        if (prev != 0xffffffffu) *reinterpret_cast<uint16_t *>(ohb + prev) = 0;
+        uint32_t off = 0xffffffffu;
+        if (valid) {
+          off = (uint32_t)(row >> 6) * (uint32_t)B * 128u + sw128_off(besti, row & 63);
+          *reinterpret_cast<uint16_t *>(ohb + off) = 0x3F80;  // bf16 1.0
+        }
+        if (ab) last_off1 = off;
+        else last_off0 = off;
+        fence_proxy_async();
+        mbar_arrive(&oh_full[ab]);
+      }
+      if (!ok) break;
+      mbar_arrive(&cnt_full[kb3]);
+      mbar_arrive(&prep_empty[cb]);
+    }
+    cp_async_wait<0>();  // no copy outlives the CTA
+    if (nan) atomicCAS(p.status, kDevOk, kDevNaN);
+  } else if (warp < 9) {
+    // --------------------------------------------------------- preparation
+    const int w6 = warp - 5, k = w6 * 32 + lane;  // this thread's dimension
+    int si = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int s = blockIdx.x; s < n_segs && ok; s += gridDim.x, ++si) {
+      const PipeSeg g = pipe_seg(p, s);
+      const int cb = si % NCB;
+      const float *gbeac = p.beacons + g.seg * B * D;
+      float *cp = cpart + (si & 1) * 4 * BM;
+      uint8_t *hb = chi + cb * kCBytes, *lb = clo + cb * kCBytes;
+      float cnext[32];
+      auto load_batch = [&](int b0) {
+        if (g.init) {
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            cnext[u] = __bfloat162float(ring[pipe_point(p, g, (int)(((int64_t)(b0 + u) * g.n_pts) / B)) + k]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) cnext[u] = gbeac[(b0 + u) * D + k];
+        }
+      };
+      load_batch(0);  // in flight while the buffer is still in use
+      ok = lanes_wait(&prep_empty[cb], ((si / NCB) & 1) ^ 1, abort_flag, p.status);
+      if (!ok) break;
+      for (int b0 = 0; b0 < B; b0 += 32) {
+        float c[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) c[u] = cnext[u];
+        if (b0 + 32 < B) load_batch(b0 + 32);
+        const uint32_t kbo = (uint32_t)(k >> 6) * (uint32_t)B * 128u;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const __nv_bfloat16 hi = __float2bfloat16_rn(c[u]);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(c[u] - __bfloat162float(hi));
+          const uint32_t off = kbo + sw128_off(b0 + u, k & 63);
+          *reinterpret_cast<__nv_bfloat16 *>(hb + off) = hi;
+          *reinterpret_cast<__nv_bfloat16 *>(lb + off) = lo;
+          c[u] = c[u] * c[u];
+        }
+        // butterfly reduce-scatter of the 32 squares over the warp's 32
+        // dimensions: lane j ends with beacon b0 + j's partial norm
+#pragma unroll
+        for (int w = 16; w >= 1; w >>= 1) {
+          const bool up = (lane & w) != 0;
+#pragma unroll
+          for (int i = 0; i < w; ++i) {
+            const float send = up ? c[i] : c[i + w];
+            const float keep = up ? c[i + w] : c[i];
+            c[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+          }
+        }
+        cp[w6 * BM + b0 + lane] = c[0];
+      }
+      fence_proxy_async();  // the beacon terms, for the MMA
+      mbar_arrive(prep_sync);
+      ok = lanes_wait(prep_sync, ph & 1, abort_flag, p.status);
+      ++ph;
+      if (!ok) break;
+      if (k < B) cn[cb * BM + k] = ((cp[k] + cp[BM + k]) + cp[2 * BM + k]) + cp[3 * BM + k];
+      mbar_arrive(&prep_full[cb]);
+    }
+  } else {
+    // -------------------------------------------------------- running mean
+    const int q = warp & 3, k = q * 32 + lane;  // this thread's dimension = its TMEM lane
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    int si = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int s = blockIdx.x; s < n_segs && ok; s += gridDim.x, ++si) {
+      const PipeSeg g = pipe_seg(p, s);
+      const int kb3 = si % 3, sb = si & 1;
+      int32_t *cntb = cnt + kb3 * BM;
+      float *gbeac = p.beacons + g.seg * B * D;
+      int32_t *gcnt = p.counts + g.seg * B;
+      __nv_bfloat16 *gs = reinterpret_cast<__nv_bfloat16 *>(p.beacons_s) + g.seg * B * D;
+      int32_t *no = nold + sb * BM;
+      // the old count and the first old values do not depend on this update's
+      // points: their loads fly while the sums are still being produced
+      const int n_old = (k < B && !g.init) ? gcnt[k] : 0;
+      float onext[32];
+      auto load_old = [&](int b0) {
+        if (g.init) {
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            onext[u] = __bfloat162float(ring[pipe_point(p, g, (int)(((int64_t)(b0 + u) * g.n_pts) / B)) + k]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) onext[u] = gbeac[(b0 + u) * D + k];
+        }
+      };
+      load_old(0);
+      ok = lanes_wait(&cnt_full[kb3], (si / 3) & 1, abort_flag, p.status) &&
+           lanes_wait(&sum_full[sb], (si >> 1) & 1, abort_flag, p.status);
+      if (!ok) break;
+      tmem_fence_after();
+      if (k < B) no[k] = n_old;
+      mbar_arrive(mean_sync);
+      ok = lanes_wait(mean_sync, ph & 1, abort_flag, p.status);
+      ++ph;
+      if (!ok) break;
+      for (int b0 = 0; b0 < B; b0 += 32) {
+        float sm[32], v[32];
+        tmem_ld32(tmem_base + lane_addr + 2 * BM + sb * BM + b0, sm);
+#pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] = onext[u];
+        if (b0 + 32 < B) load_old(b0 + 32);
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const int b = b0 + u;
+          const int m = cntb[b], n = no[b];
+          float x = v[u];
+          if (m > 0) x = ((float)n * x + sm[u]) / (float)(n + m);
+          gbeac[b * D + k] = x;
+          gs[b * D + k] = __float2bfloat16_rn(x);
+        }
+      }
+      tmem_fence_before();
+      mbar_arrive(&sum_empty[sb]);
+      // every thread has read all counts before they are zeroed
+      mbar_arrive(mean_sync);
+      ok = lanes_wait(mean_sync, ph & 1, abort_flag, p.status);
+      ++ph;
+      if (!ok) break;
+      if (k < B) {
+        const int m = cntb[k];
+        gcnt[k] = no[k] + m;
+        p.trig[g.seg * B + k] = (float)m / (float)g.n_pts;
+        cntb[k] = 0;
+      }
+      mbar_arrive(&cnt_empty[kb3]);
+    }
+  }
+  tmem_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tmem_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(4 * BM));
+  }
+}
+
+template <int BM, int NXS, int NCB, int DA>
+cudaError_t launch_pipe(const BeaconUpdateParams &p, int n_segs, cudaStream_t s) {
+  const size_t smem = 1024 + (size_t)NXS * 32768 + 2 * (size_t)NCB * BM * 256 + 2 * (size_t)BM * 256 +
+                      sizeof(float) * ((size_t)NCB * BM + 8 * BM) + sizeof(int32_t) * (3 * (size_t)BM + 2 * BM) +
+                      8 * (2 * NXS + 2 * NCB + 6 + 12 + 3) + 16;  // barriers, TMEM slot, abort flag
+  cudaError_t e = cudaFuncSetAttribute(beacon_update_pipe_kernel<BM, NXS, NCB, DA>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = n_segs < sms ? n_segs : sms;
+  beacon_update_pipe_kernel<BM, NXS, NCB, DA><<<grid, kPipeThreads, smem, s>>>(p, n_segs);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool beacon_update_tc_supported(int d, int B, int dtype) {
@@ -355,6 +843,9 @@ cudaError_t launch_beacon_update_tc(const BeaconUpdateParams &p, int n_req, cuda
   // point tile, c_hi/c_lo tiles, one-hot tile, cn + cpart[4] + cnt (6 words per
   // beacon), barrier/slot/flag; TMEM: assignment columns then 128 per half
   const size_t smem = 1024 + 32768 + (size_t)p.B * 512 + 32768 + (size_t)p.B * 4 * 6 + 64;
+  const int n_segs = n_req * p.layers * p.hkv;
+  if (p.B <= 64) return launch_pipe<64, 3, 2, 2>(p, n_segs, s);
+  if (p.B <= 128) return launch_pipe<128, 2, 1, 1>(p, n_segs, s);
   const uint32_t cols = p.B <= 128 ? 256u : 512u;
   cudaError_t e = cudaFuncSetAttribute(beacon_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
