@@ -29,19 +29,16 @@
 // page q (a page holds 16 keys x 256 B contiguous; that map covers the pool
 // as rows of 128 bf16).  The number of boxes, not their bytes, limited the
 // key stream; warp 1 issues the MMAs (one elected lane) and commits them to
-// mbarriers; the remaining warps run the epilogue in groups of four, group g
-// taking every kEpiGroups-th accumulator item (tcgen05.ld of 64 columns at a
-// time; sums and maxima in 8 independent partials; the per-beacon partial
-// (max, sum) of the groups merged once per segment).
+// mbarriers; warps 2-9 run the epilogue in two groups of four, group g taking
+// the tiles whose accumulator is in TMEM buffers of parity g (tcgen05.ld of
+// 64 columns at a time; sums and maxima in 8 independent partials; the
+// per-beacon partial (max, sum) of the groups merged once per segment).
 // Pass 1 adds a full 64-column chunk as sum 2^(u - m) against the running
 // reference m with no max pass first; only a chunk whose sum would pass
 // 2^64 (a new maximum far above m) or a partial chunk takes the max-then-
 // rescale step.  Key tiles rotate through 4 shared-memory stages; the
-// accumulators through four 128-column TMEM slots: with more than 128
-// beacons a pass-1 tile is issued as two 64-key items of one slot each and a
-// pass-2 tile as one item over two slots (one per 128-beacon half), so the
-// MMA warp can run ahead of the epilogue by the same four slots at every
-// beacon count.  No load uses cluster multicast.
+// accumulators through four 128-column TMEM buffers (at most 128 beacons)
+// or two of 256.  No load uses cluster multicast.
 // Every mbarrier wait is bounded (2 s of %globaltimer): on expiry the kernel
 // records KVC_ERR_DEVICE_TIMEOUT in the status word, the other roles see the
 // abort flag and leave, and TMEM is released before the CTA exits.
@@ -62,12 +59,8 @@ namespace kvc {
 namespace {
 
 constexpr int kTileKeys = 128;
-#ifndef KVC_TC_EPI_GROUPS
-#define KVC_TC_EPI_GROUPS 2
-#endif
-constexpr int kEpiGroups = KVC_TC_EPI_GROUPS;  // groups of 4 warps; item i goes to group i % kEpiGroups
-constexpr int kEpiWarps = 4 * kEpiGroups;
-constexpr int kThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, then the epilogue warps
+constexpr int kEpiWarps = 8;   // two groups of 4: group g drains accumulator buffer g
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr uint32_t kTmemCols = 512;
 
 struct TcParams {
@@ -90,11 +83,12 @@ struct SegGeom {
   int nres;        // pass-2 tiles still resident in their pass-1 stages
   // tile index of item t of the segment's sequence: pass 1 in order, then
   // pass 2 starting with the resident tiles (the last nres of pass 1), then
-  // the remaining generated tiles in order
+  // the remaining generated tiles from the last down, so that the tiles pass
+  // 1 loaded most recently, the likeliest to still be in L2, come first
   __device__ __forceinline__ int tile_of(int t) const {
     if (t < n1) return t;
     const int u = t - n1;
-    return u < nres ? n1 - nres + u : t2 + (u - nres);
+    return u < nres ? n1 - nres + u : n1 - 1 - u;
   }
 };
 template <int S>
@@ -136,14 +130,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = smem_align<1024>(smem_raw);
   constexpr uint32_t kCBytes = CROWS * 256;          // beacon tile: CROWS rows x 128 bf16
   constexpr uint32_t kTileBytes = kTileKeys * 256;   // 32 KB
-  // TMEM accumulator slots: 4 of 128 columns.  With at most 128 beacons a
-  // tile's products fill one slot.  With more (kSplit) a pass-1 tile is two
-  // items of 64 keys, each one slot (beacon half h in columns [64h, 64h+64)),
-  // and a pass-2 tile is one item of two consecutive slots (beacon half h in
-  // the h-th), so the MMA warp still runs up to four slots ahead of the
-  // epilogue.  Items go round-robin to the epilogue groups.
-  constexpr bool kSplit = CROWS > 128;
-  constexpr int NACC = 4;
+  // TMEM accumulator buffers: 4 of 128 columns when a tile's products fit in
+  // 128 columns (at most 128 beacons), else 2 of 256; the epilogue group g
+  // drains the buffers b with b % 2 == g
+  constexpr int NACC = CROWS <= 128 ? 4 : 2;
   constexpr uint32_t ACOLS = kTmemCols / NACC;
   uint8_t *cbuf = smem;                              // [NCB][2 K-halves][CROWS][128 B]
   uint8_t *kbuf = smem + NCB * kCBytes;              // [kStages][2][128][128 B]
@@ -155,8 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(epi_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *lse2 = reinterpret_cast<float *>(tmem_slot + 4);  // [2][256]
-  float *part = lse2 + 512;                                 // [2 kEpiGroups][2][256] partial (m, sum)
-  float *wts2 = part + 2 * kEpiGroups * 2 * 256;            // [2][256] trigger shares
+  float *part = lse2 + 512;                                 // [4][2][256] partial (m, sum)
+  float *wts2 = part + 4 * 2 * 256;                         // [2][256] trigger shares
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -272,75 +262,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      uint32_t it = 0, acc_it = 0;  // key tiles; accumulator slots taken
+      uint32_t it = 0, acc_it = 0;
       int si = 0;
-      const uint32_t idesc1 = idesc_bf16_f32(128, kSplit ? kTileKeys / 2 : kTileKeys);
-      const uint32_t idesc2 = idesc_bf16_f32(128, kSplit ? 128 : B);
-      const uint32_t idesc2b = idesc_bf16_f32(128, kSplit ? B - 128 : B);  // second beacon half
+      const uint32_t idesc1 = idesc_bf16_f32(128, kTileKeys);
+      const uint32_t idesc2 = idesc_bf16_f32(128, B);
       bool ok = true;
-      // slot a % NACC is free once the epilogue drained its previous use
-      auto take = [&](uint32_t a) {
-        return mbar_wait(&acc_empty[a % NACC], ((a / NACC) & 1) ^ 1, abort_flag, p.status);
-      };
       for (int s = blockIdx.x; s < p.n_segs && ok; s += gridDim.x, ++si) {
         const SegGeom g = seg_geom<kStages>(p, s);
         const int cb = si % NCB;
         ok = mbar_wait(&c_full[cb], (si / NCB) & 1, abort_flag, p.status);
         if (!ok) break;
         const uint32_t c_addr = smem_u32(cbuf + cb * kCBytes);
-        for (int t = 0; t < g.n1 + g.n2; ++t, ++it) {
-          const int st = it % kStages;
-          ok = mbar_wait(&full[st], (it / kStages) & 1, abort_flag, p.status);
+        for (int t = 0; t < g.n1 + g.n2; ++t, ++it, ++acc_it) {
+          const int st = it % kStages, buf = acc_it % NACC;
+          ok = mbar_wait(&full[st], (it / kStages) & 1, abort_flag, p.status) &&
+               mbar_wait(&acc_empty[buf], ((acc_it / NACC) & 1) ^ 1, abort_flag, p.status);
           if (!ok) break;
+          tmem_fence_after();
           const uint32_t k_addr = smem_u32(kbuf + st * kTileBytes);
-          if (t < g.n1 && !kSplit) {
-            ok = take(acc_it);
-            if (!ok) break;
-            tmem_fence_after();
-            const uint32_t d = tmem_base + (acc_it % NACC) * ACOLS;
-            for (int kb = 0; kb < 2; ++kb)
-              for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t a = sw128_desc(c_addr + kb * CROWS * 128 + ks * 32);
-                const uint64_t b = sw128_desc(k_addr + kb * kTileKeys * 128 + ks * 32);
-                umma(d, a, b, idesc1, (kb | ks) != 0);
-              }
-            umma_commit(&acc_full[acc_it % NACC]);
-            ++acc_it;
-          } else if (t < g.n1) {
-            for (int kh = 0; kh < 2 && ok; ++kh) {
-              ok = take(acc_it);
-              if (!ok) break;
-              tmem_fence_after();
-              const uint32_t d = tmem_base + (acc_it % NACC) * ACOLS;
-              for (int half = 0; half < 2; ++half)
-                for (int kb = 0; kb < 2; ++kb)
-                  for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t a = sw128_desc(c_addr + kb * CROWS * 128 + half * 128 * 128 + ks * 32);
-                    const uint64_t b = sw128_desc(k_addr + kb * kTileKeys * 128 + kh * 64 * 128 + ks * 32);
-                    umma(d + half * 64, a, b, idesc1, (kb | ks) != 0);
-                  }
-              umma_commit(&acc_full[acc_it % NACC]);
-              ++acc_it;
-            }
-            if (!ok) break;
-          } else {
-            const int nslot = kSplit ? 2 : 1;
-            ok = take(acc_it) && (nslot == 1 || take(acc_it + 1));
-            if (!ok) break;
-            tmem_fence_after();
-            for (int half = 0; half < nslot; ++half) {
-              const uint32_t d = tmem_base + ((acc_it + half) % NACC) * ACOLS;
+          const uint32_t d = tmem_base + buf * ACOLS;
+          if (t < g.n1) {
+            for (int half = 0; half * 128 < B; ++half)
               for (int kb = 0; kb < 2; ++kb)
                 for (int ks = 0; ks < 4; ++ks) {
-                  const uint64_t a = sw128_desc(k_addr + kb * kTileKeys * 128 + ks * 32);
-                  const uint64_t b = sw128_desc(c_addr + kb * CROWS * 128 + half * 128 * 128 + ks * 32);
-                  umma(d, a, b, half ? idesc2b : idesc2, (kb | ks) != 0);
+                  const uint64_t a = sw128_desc(c_addr + kb * CROWS * 128 + half * 128 * 128 + ks * 32);
+                  const uint64_t b = sw128_desc(k_addr + kb * kTileKeys * 128 + ks * 32);
+                  umma(d + half * 128, a, b, idesc1, (kb | ks) != 0);
                 }
-            }
-            for (int half = 0; half < nslot; ++half) umma_commit(&acc_full[(acc_it + half) % NACC]);
-            acc_it += nslot;
+          } else {
+            for (int kb = 0; kb < 2; ++kb)
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t a = sw128_desc(k_addr + kb * kTileKeys * 128 + ks * 32);
+                const uint64_t b = sw128_desc(c_addr + kb * CROWS * 128 + ks * 32);
+                umma(d, a, b, idesc2, (kb | ks) != 0);
+              }
           }
           umma_commit(&empty[st]);
+          umma_commit(&acc_full[buf]);
         }
         if (!ok) break;
         umma_commit(&c_empty[cb]);
@@ -350,19 +308,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    // Group grp (warps 2 + 4 grp .. 5 + 4 grp) handles the items i with
-    // i % kEpiGroups == grp; each warp reads the TMEM lane
+    // Group grp (warps 2-5 or 6-9) handles the tiles whose accumulator sits
+    // in buffer grp, i.e. every other tile; each warp reads the TMEM lane
     // quarter (warp % 4) it may access.
     const int ew = warp - 2, grp = ew >> 2;
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int row = q * 32 + lane;          // TMEM lane = D row
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     const int copy = dup ? (row >> 6) : 0;  // warp-uniform
-    const int col_lo = dup ? copy * 64 : 0, ncols = (dup || kSplit) ? 64 : kTileKeys;
-    const int nslot = kEpiGroups * (dup ? 2 : 1);  // partials per beacon: groups x copies
+    const int col_lo = dup ? copy * 64 : 0, ncols = dup ? 64 : kTileKeys;
+    const int nslot = dup ? 4 : 2;          // partials per beacon: groups x copies
     const int slot = grp * (dup ? 2 : 1) + copy;
     const float alpha = p.alpha;
-    uint32_t acc_it = 0, item = 0, epi_ph = 0;  // accumulator slots, items (alternating groups)
+    uint32_t acc_it = 0, epi_ph = 0;
     int si = 0;
     bool ok = true;
     for (int s = blockIdx.x; s < p.n_segs && ok; s += gridDim.x, ++si) {
@@ -371,10 +329,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float *w_buf = wts2 + (si & 1) * 256;
       // pass 1: per-beacon online log2-sum-exp2 over this group's tiles
       float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
-      for (int t = 0; t < g.n1 && ok; ++t)
-       for (int kh = 0; kh < (kSplit ? 2 : 1); ++kh, ++acc_it, ++item) {
+      for (int t = 0; t < g.n1; ++t, ++acc_it) {
         const int buf = acc_it % NACC;
-        if (item % kEpiGroups != (uint32_t)grp) continue;
+        if ((buf & 1) != grp) continue;
         ok = warp_wait(&acc_full[buf], (acc_it / NACC) & 1, abort_flag, p.status);
         if (!ok) break;
         tmem_fence_after();
@@ -387,15 +344,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           float &sum = half ? s1 : s0;
           for (int c0 = col_lo; c0 < col_lo + ncols; c0 += 64) {
             float v[64];
-            tmem_ld64(tmem_base + lane_addr + buf * ACOLS + (kSplit ? half * 64 : half * 128 + c0), v);
+            tmem_ld64(tmem_base + lane_addr + buf * ACOLS + half * 128 + c0, v);
             if (half == nhalf - 1 && c0 + 64 >= col_lo + ncols) {
-              // the item's last load has landed in registers: hand the
-              // slot back to the MMA warp before the arithmetic
+              // the tile's last load has landed in registers: hand the
+              // buffer back to the MMA warp before the arithmetic
               tmem_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&acc_empty[buf]);
             }
-            const int nv = min(64, nvalid - (kSplit ? kh * 64 : c0));
+            const int nv = min(64, nvalid - c0);
             if (!mine || nv <= 0) continue;
             if (nv == 64 && m != -INFINITY) {
               // full chunk against the running reference m, with no max
@@ -481,11 +438,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++epi_ph;
       if (!ok) break;
       // pass 2: per-key max over beacons of u - lse2 (this group's tiles)
-      for (int t = 0; t < g.n2; ++t, acc_it += (kSplit ? 2 : 1), ++item) {
-        const int buf = acc_it % NACC, buf2 = (acc_it + 1) % NACC;
-        if (item % kEpiGroups != (uint32_t)grp) continue;
-        ok = warp_wait(&acc_full[buf], (acc_it / NACC) & 1, abort_flag, p.status) &&
-             (!kSplit || warp_wait(&acc_full[buf2], ((acc_it + 1) / NACC) & 1, abort_flag, p.status));
+      for (int t = 0; t < g.n2; ++t, ++acc_it) {
+        const int buf = acc_it % NACC;
+        if ((buf & 1) != grp) continue;
+        ok = warp_wait(&acc_full[buf], (acc_it / NACC) & 1, abort_flag, p.status);
         if (!ok) break;
         tmem_fence_after();
         float bm[8];
@@ -495,18 +451,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 8; ++i) bm[i] = trig ? 0.f : -INFINITY;
         for (int c0 = 0; c0 < B; c0 += 64) {
           float v[64];
-          // beacons [0, 128) in the first slot, [128, B) in the second (kSplit)
-          const uint32_t col = (kSplit && c0 >= 128) ? buf2 * ACOLS + (c0 - 128) : buf * ACOLS + c0;
-          tmem_ld64(tmem_base + lane_addr + col, v);
-          if (c0 + 64 >= (kSplit ? min(B, 128) : B) && c0 < 128) {  // the first slot's last load
+          tmem_ld64(tmem_base + lane_addr + buf * ACOLS + c0, v);
+          if (c0 + 64 >= B) {  // the tile's last load: hand the buffer back
             tmem_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
-          }
-          if (kSplit && c0 + 64 >= B && c0 >= 128) {  // the second slot's last load
-            tmem_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf2]);
           }
           const float4 *l4 = reinterpret_cast<const float4 *>(lse_buf + c0);
           if (trig) {
@@ -598,7 +547,7 @@ template <int CROWS, int NCB, int kStages>
 cudaError_t launch(const CUtensorMap &km, const CUtensorMap &cm, const CUtensorMap &km4, const TcParams &tp,
                    cudaStream_t s) {
   const size_t smem = 1024 + (size_t)NCB * CROWS * 256 + (size_t)kStages * kTileKeys * 256 + 256 +
-                      2 * 256 * 4 + 2 * kEpiGroups * 2 * 256 * 4 + 2 * 256 * 4;
+                      2 * 256 * 4 + 4 * 2 * 256 * 4 + 2 * 256 * 4;
   cudaError_t e = cudaFuncSetAttribute(beacon_score_tc_kernel<CROWS, NCB, kStages>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -363,7 +363,9 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
 //   warps 5-8   preparation: the next segment's beacons as bf16 hi/lo terms
 //               (swizzled, the B operand of the assignment) and their fp32
 //               squared norms;
-//   warps 9-12  running mean: one dimension per thread, over every beacon.
+//   warps 9-12  running mean: one dimension per thread, over every beacon,
+//               (n c + sum) * (1 / (n + m)) with the reciprocal taken once
+//               per beacon.
 // The sums are D[dim][beacon] = X^T OH, with the point tile read as an
 // MN-major A operand (dimensions on M, its 64-dimension blocks 16 KB apart)
 // and the one-hot tile OH [beacon rows x point columns] as a K-major B
@@ -436,8 +438,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   float *cn = reinterpret_cast<float *>(oh + 2 * kOHBytes);     // [NCB][BM] squared norms
   float *cpart = cn + NCB * BM;                                   // [2][4][BM] per-warp partial norms
   int32_t *cnt = reinterpret_cast<int32_t *>(cpart + 8 * BM);    // [3][BM] this update's counts
-  int32_t *nold = cnt + 3 * BM;                                   // [2][BM] counts before the update
-  uint64_t *bars = reinterpret_cast<uint64_t *>(nold + 2 * BM);
+  float *mfac = reinterpret_cast<float *>(cnt + 3 * BM);          // [2][2][BM] old count n, 1/(n+m) or 0
+  uint64_t *bars = reinterpret_cast<uint64_t *>(mfac + 4 * BM);
   uint64_t *x_full = bars, *x_empty = x_full + NXS;
   uint64_t *prep_full = x_empty + NXS, *prep_empty = prep_full + NCB;
   uint64_t *cnt_full = prep_empty + NCB, *cnt_empty = cnt_full + 3;
@@ -750,7 +752,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       float *gbeac = p.beacons + g.seg * B * D;
       int32_t *gcnt = p.counts + g.seg * B;
       __nv_bfloat16 *gs = reinterpret_cast<__nv_bfloat16 *>(p.beacons_s) + g.seg * B * D;
-      int32_t *no = nold + sb * BM;
+      float *nf = mfac + sb * 2 * BM, *inv = nf + BM;
       // the old count and the first old values do not depend on this update's
       // points: their loads fly while the sums are still being produced
       const int n_old = (k < B && !g.init) ? gcnt[k] : 0;
@@ -770,7 +772,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
            lanes_wait(&sum_full[sb], (si >> 1) & 1, abort_flag, p.status);
       if (!ok) break;
       tmem_fence_after();
-      if (k < B) no[k] = n_old;
+      // per beacon: n and 1/(n + m), or 0 when no point joined it (unchanged)
+      if (k < B) {
+        const int m = cntb[k];
+        nf[k] = (float)n_old;
+        inv[k] = m > 0 ? 1.f / (float)(n_old + m) : 0.f;
+      }
       mbar_arrive(mean_sync);
       ok = lanes_wait(mean_sync, ph & 1, abort_flag, p.status);
       ++ph;
@@ -784,9 +791,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
           const int b = b0 + u;
-          const int m = cntb[b], n = no[b];
-          float x = v[u];
-          if (m > 0) x = ((float)n * x + sm[u]) / (float)(n + m);
+          const float iv = inv[b];
+          const float x = iv != 0.f ? fmaf(nf[b], v[u], sm[u]) * iv : v[u];
           gbeac[b * D + k] = x;
           gs[b * D + k] = __float2bfloat16_rn(x);
         }
@@ -800,7 +806,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       if (!ok) break;
       if (k < B) {
         const int m = cntb[k];
-        gcnt[k] = no[k] + m;
+        gcnt[k] = n_old + m;
         p.trig[g.seg * B + k] = (float)m / (float)g.n_pts;
         cntb[k] = 0;
       }
@@ -818,7 +824,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 template <int BM, int NXS, int NCB, int DA>
 cudaError_t launch_pipe(const BeaconUpdateParams &p, int n_segs, cudaStream_t s) {
   const size_t smem = 1024 + (size_t)NXS * 32768 + 2 * (size_t)NCB * BM * 256 + 2 * (size_t)BM * 256 +
-                      sizeof(float) * ((size_t)NCB * BM + 8 * BM) + sizeof(int32_t) * (3 * (size_t)BM + 2 * BM) +
+                      sizeof(float) * ((size_t)NCB * BM + 8 * BM + 4 * BM) + sizeof(int32_t) * 3 * (size_t)BM +
                       8 * (2 * NXS + 2 * NCB + 6 + 12 + 3) + 16;  // barriers, TMEM slot, abort flag
   cudaError_t e = cudaFuncSetAttribute(beacon_update_pipe_kernel<BM, NXS, NCB, DA>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

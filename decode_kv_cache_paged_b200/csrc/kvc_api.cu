@@ -30,7 +30,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
   size_t bt, len, prompt, pos, qring, beacons, beacons_s, counts, trig, scores, lse, status, counters,
-      stage, attn, ranks, first, total, stage_slot;
+      stage, attn, total, stage_slot;
 };
 
 // Split partials of the decode attention: room for this many splits of one layer.
@@ -92,12 +92,6 @@ Layout make_layout(const kvc_config &c) {
   L.stage_slot = align_up(R * 16 + R * maxp * 8 + R * 8 + 1024, 256);
   L.stage = take(L.stage_slot * kStageSlots);
   L.attn = take(R * Hq * (d + 2) * 4 * (size_t)kAttnSplits);
-  // rank maps of the split select/copy launches (segments of more than
-  // kSplitMinN candidates), two layers' worth so that one layer's select can
-  // run while the previous layer's copy reads the other
-  const bool split = c.max_seq_len > kSplitMinN;
-  L.ranks = take(split ? 2 * R * H * (size_t)c.max_seq_len * 2 : 0);
-  L.first = take(split ? 2 * R * H * 4 : 0);
   L.total = off;
   return L;
 }
@@ -130,12 +124,6 @@ struct kvc_ctx {
   std::vector<uint8_t> h_unordered;  // a hole-filling round left slots out of position order
   std::vector<int32_t> free_pages;
   int64_t round = 0;
-  // split select/copy rounds: a second stream for the selects, its events,
-  // and the two rank-map buffers in the workspace
-  cudaStream_t side = nullptr;
-  cudaEvent_t fork_ev = nullptr, sel_ev[2] = {}, copy_ev[2] = {};
-  uint16_t *d_ranks = nullptr;
-  int32_t *d_first = nullptr;
   int score_impl = 0;
   int update_impl = 0;
   int es = 2, row_bytes = 0, G = 1, maxp = 0, num_sms = 148;
@@ -311,8 +299,6 @@ kvc_status kvc_create(const kvc_config *cfg, void *k_pool, void *v_pool, void *w
   c->d_counters = reinterpret_cast<unsigned long long *>(c->ws + lay.counters);
   c->d_stage = c->ws + lay.stage;
   c->d_attn = reinterpret_cast<float *>(c->ws + lay.attn);
-  c->d_ranks = reinterpret_cast<uint16_t *>(c->ws + lay.ranks);
-  c->d_first = reinterpret_cast<int32_t *>(c->ws + lay.first);
   if (cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
     cudaGetLastError();
     c->num_sms = 148;
@@ -336,9 +322,6 @@ kvc_status kvc_create(const kvc_config *cfg, void *k_pool, void *v_pool, void *w
       if (ev) cudaEventDestroy(ev);
     for (auto &ev : c->ev)
       if (ev) cudaEventDestroy(ev);
-    for (cudaEvent_t ev : {c->fork_ev, c->sel_ev[0], c->sel_ev[1], c->copy_ev[0], c->copy_ev[1]})
-      if (ev) cudaEventDestroy(ev);
-    if (c->side) cudaStreamDestroy(c->side);
     if (c->h_stage) cudaFreeHost(c->h_stage);
     delete c;
     return s;
@@ -350,13 +333,6 @@ kvc_status kvc_create(const kvc_config *cfg, void *k_pool, void *v_pool, void *w
       return cleanup(e, "cudaEventCreate");
   for (auto &ev : c->ev)
     if ((e = cudaEventCreate(&ev)) != cudaSuccess) return cleanup(e, "cudaEventCreate");
-  if (cfg->max_seq_len > kSplitMinN) {
-    if ((e = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking)) != cudaSuccess)
-      return cleanup(e, "cudaStreamCreate(side)");
-    for (cudaEvent_t *ev : {&c->fork_ev, &c->sel_ev[0], &c->sel_ev[1], &c->copy_ev[0], &c->copy_ev[1]})
-      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess)
-        return cleanup(e, "cudaEventCreate");
-  }
   // device state: block tables -1, lengths 0, position map -1, beacon counts 0
   if ((e = cudaMemsetAsync(c->d_bt, 0xff, (size_t)R * c->maxp * 4, c->stream)) != cudaSuccess ||
       (e = cudaMemsetAsync(c->d_len, 0, (size_t)R * 4, c->stream)) != cudaSuccess ||
@@ -375,12 +351,6 @@ kvc_status kvc_destroy(kvc_ctx *ctx) {
   cudaStreamSynchronize(ctx->stream);
   for (auto &ev : ctx->stage_ev) cudaEventDestroy(ev);
   for (auto &ev : ctx->ev) cudaEventDestroy(ev);
-  if (ctx->side) {
-    cudaStreamSynchronize(ctx->side);
-    cudaStreamDestroy(ctx->side);
-    for (cudaEvent_t ev : {ctx->fork_ev, ctx->sel_ev[0], ctx->sel_ev[1], ctx->copy_ev[0], ctx->copy_ev[1]})
-      cudaEventDestroy(ev);
-  }
   cudaFreeHost(ctx->h_stage);
   delete ctx;
   return KVC_OK;
@@ -705,19 +675,8 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
   sp.round = (uint64_t)ctx->round;
   const int mode = selector == KVC_SEL_RANDOM ? kModeRandom
                    : selector == KVC_SEL_RANDOM_SHARED ? kModeRandomShared : kModeScores;
-  sp.layer0 = 0;
-  sp.nlayers = c.num_layers;
-  // buckets: candidate counts up to 2^k.  Buckets of more than kSplitMinN
-  // candidates with order-preserving compaction run as a select launch and a
-  // copy launch per layer: the selects on the side stream, the copies on the
-  // context's stream, so that layer l+1's select (arithmetic: draws, radix
-  // select, ranks) overlaps layer l's copy (HBM).  Rank buffers alternate by
-  // layer; a select reuses one only after the copy two layers back has read it.
+  // buckets: candidate counts up to 2^k
   size_t i0 = 0;
-  int split_layers = 0;  // split (bucket, layer) launches so far this round
-  // the selects wait for what precedes the round's selection (the scores),
-  // not for the fused launches of the smaller buckets
-  if (ctx->side && !segs.empty()) KVC_CUDA(ctx, cudaEventRecord(ctx->fork_ev, ctx->stream));
   while (i0 < segs.size()) {
     int cap = 1024;
     while (cap < segs[i0].L - segs[i0].P) cap *= 2;
@@ -729,31 +688,9 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
     }
     const int max_n = segs[i1 - 1].L - segs[i1 - 1].P;
     sp.segs = d_segs + i0;
-    const int n = (int)(i1 - i0);
-    if (max_n > kSplitMinN && o.compaction == KVC_COMPACT_ORDERED && ctx->side) {
-      if (split_layers == 0) KVC_CUDA(ctx, cudaStreamWaitEvent(ctx->side, ctx->fork_ev, 0));
-      for (int l = 0; l < c.num_layers; ++l, ++split_layers) {
-        const int b = split_layers & 1;
-        SelectCompactParams lp = sp;
-        lp.layer0 = l;
-        lp.nlayers = 1;
-        lp.ranks = ctx->d_ranks + (size_t)b * R * c.num_kv_heads * c.max_seq_len;
-        lp.first_evicted = ctx->d_first + (size_t)b * R * c.num_kv_heads;
-        if (split_layers >= 2) KVC_CUDA(ctx, cudaStreamWaitEvent(ctx->side, ctx->copy_ev[b], 0));
-        e = launch_select_ranks(lp, mode, n, max_n, ctx->side);
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "select_ranks");
-        KVC_CUDA(ctx, cudaEventRecord(ctx->sel_ev[b], ctx->side));
-        KVC_CUDA(ctx, cudaStreamWaitEvent(ctx->stream, ctx->sel_ev[b], 0));
-        e = launch_compact_copy(lp, n, max_m, ctx->stream);
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "compact_copy");
-        KVC_CUDA(ctx, cudaEventRecord(ctx->copy_ev[b], ctx->stream));
-        st.launches += 2;
-      }
-    } else {
-      e = launch_select_compact(sp, mode, n, max_n, max_m, ctx->stream);
-      if (e != cudaSuccess) return cuda_fail(ctx, e, "select_compact");
-      st.launches += 1;
-    }
+    e = launch_select_compact(sp, mode, (int)(i1 - i0), max_n, max_m, ctx->stream);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "select_compact");
+    st.launches += 1;
     i0 = i1;
   }
   if (timed) KVC_CUDA(ctx, cudaEventRecord(ctx->ev[2], ctx->stream));

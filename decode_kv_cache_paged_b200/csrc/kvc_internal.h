@@ -44,14 +44,6 @@ struct SelectCompactParams {
   int32_t block;  // positions per Philox draw (random selectors)
   int32_t flags;  // kScTieByPos | kScHoleFill
   uint64_t seed, round;
-  // layers [layer0, layer0 + nlayers) of each listed request take part in a
-  // launch (CTA b: head b % hkv, layer layer0 + (b / hkv) % nlayers)
-  int32_t layer0, nlayers;
-  // split rounds: the select launch writes each segment's first evicted
-  // candidate and its rank -> candidate map here, the copy launch reads them
-  // ([R][hkv] and [R][hkv][max_seq], this launch's layer only)
-  int32_t *first_evicted;
-  uint16_t *ranks;
 };
 
 // SelectCompactParams::flags
@@ -126,14 +118,6 @@ cudaError_t launch_wait_timeout_probe(int32_t *status, uint32_t limit_ms, cudaSt
 bool decode_attention_supported(int dtype, int head_dim, int G);
 cudaError_t launch_decode_attention(const DecodeAttnParams &p, int head_dim, int dtype, int G, int *launches,
                                     cudaStream_t s);
-// A large-candidate round split in two launches over one layer: the select
-// (scores, threshold, ranks; written to p.ranks / p.first_evicted) and the
-// in-place copy that reads them, so that one layer's select can run beside
-// another layer's copy on a second stream.  Order-preserving compaction only.
-cudaError_t launch_select_ranks(const SelectCompactParams &p, int mode, int n_seg_req, int max_n, cudaStream_t s);
-cudaError_t launch_compact_copy(const SelectCompactParams &p, int n_seg_req, int max_m, cudaStream_t s);
-// Candidate counts above this use the split launches for order-preserving rounds.
-constexpr int kSplitMinN = 4096;
 cudaError_t launch_select_compact(const SelectCompactParams &p, int mode, int n_seg_req,
                                   int max_n, int max_m, cudaStream_t s);
 cudaError_t launch_beacon_update(const BeaconUpdateParams &p, int n_req, cudaStream_t s);

@@ -214,57 +214,11 @@ __device__ __forceinline__ int block_scan_each(int lo, int hi, Pred pred, Fn fn,
   return tot;
 }
 
-// In-place, order-preserving copy of ranks [q0, M): rank q moves from slot
-// P + src_of_rank[q] to slot P + q (K row, V row and position entry).  Each
-// chunk is read with 16-byte vector loads into registers, the CTA
-// synchronises, then writes.  A chunk only writes slots below its own highest
-// source slot and the next chunk only reads slots above it, so one barrier
-// per chunk makes the in-place move safe while the loads of chunk c+1
-// overlap the stores of chunk c.
-template <int NT, int kUnroll, class RowOf>
-__device__ __forceinline__ void copy_ranks(const SelectCompactParams &p, int P, int M, int q0,
-                                           const uint16_t *src_of_rank, RowOf row_of) {
-  const int tid = threadIdx.x;
-  const int vpr = p.row_bytes >> 4;  // 16-byte vectors per row
-  const int rows_per_pass = NT / vpr;
-  const int my_row = tid / vpr, my_vec = tid - (tid / vpr) * vpr;
-  const bool active = my_row < rows_per_pass;
-  const int64_t rb = p.row_bytes;
-#pragma unroll 1
-  for (int base = q0; base < M; base += rows_per_pass * kUnroll) {
-    uint4 kr[kUnroll], vr[kUnroll];
-    int pr[kUnroll];
-    int64_t drow[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int q = base + u * rows_per_pass + my_row;
-      drow[u] = -1;
-      if (active && q < M) {
-        const int64_t srow = row_of(P + src_of_rank[q]);
-        drow[u] = row_of(P + q);
-        kr[u] = *reinterpret_cast<const uint4 *>(p.k_pool + srow * rb + my_vec * 16);
-        vr[u] = *reinterpret_cast<const uint4 *>(p.v_pool + srow * rb + my_vec * 16);
-        if (my_vec == 0) pr[u] = p.pos_map[srow];
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (drow[u] >= 0) {
-        *reinterpret_cast<uint4 *>(p.k_pool + drow[u] * rb + my_vec * 16) = kr[u];
-        *reinterpret_cast<uint4 *>(p.v_pool + drow[u] * rb + my_vec * 16) = vr[u];
-        if (my_vec == 0) p.pos_map[drow[u]] = pr[u];
-      }
-    }
-  }
-  if (tid == 0 && M > q0) atomicAdd(p.counters, (unsigned long long)(M - q0));
-}
-
-template <int NT, int MODE, int kUnroll, int VAR, bool SPLIT>
+template <int NT, int MODE, int kUnroll, int VAR>
 __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams p, int keys_cap) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint32_t *keys = reinterpret_cast<uint32_t *>(smem);                  // [keys_cap]
-  uint16_t *src_of_rank = reinterpret_cast<uint16_t *>(keys + keys_cap);  // [keys_cap] (fused launches)
+  uint16_t *src_of_rank = reinterpret_cast<uint16_t *>(keys + keys_cap);  // [keys_cap]
   __shared__ uint32_t hist[256];
   __shared__ uint32_t bcast[4];
   __shared__ uint32_t cand[kFinish];
@@ -273,16 +227,13 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x % p.hkv;
-  const int l = p.layer0 + (blockIdx.x / p.hkv) % p.nlayers;
-  const SegDesc sd = p.segs[blockIdx.x / (p.hkv * p.nlayers)];
+  const int l = (blockIdx.x / p.hkv) % p.layers;
+  const SegDesc sd = p.segs[blockIdx.x / (p.hkv * p.layers)];
   const int r = sd.req, P = sd.P, M = sd.M;
   const int N = sd.L - P;
   const int32_t *bt = p.block_table + (int64_t)r * p.bt_stride;
   const int64_t layer_page0 = (int64_t)l * p.num_pages;
   const int64_t seg_flat = ((int64_t)r * p.layers + l) * p.hkv + h;
-  // rank -> candidate map: shared memory when this launch also copies, the
-  // global rank buffer of the split launches otherwise
-  uint16_t *sor = SPLIT ? p.ranks + ((int64_t)r * p.hkv + h) * p.max_seq : src_of_rank;
   // global row index (also the position-map index) of slot s of this segment
   auto row_of = [&](int s) -> int64_t {
     return ((layer_page0 + bt[s >> 4]) * p.hkv + h) * kPage + (s & (kPage - 1));
@@ -379,7 +330,7 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
         const int eq_before = off_eq + __popc(meq & lt_mask);
         const bool kept = gt || (eq && eq_before < need);
         if (kept) {
-          sor[gt_before + min(eq_before, need)] = (uint16_t)j;
+          src_of_rank[gt_before + min(eq_before, need)] = (uint16_t)j;
         } else if (valid) {
           atomicMin(&first_evicted, j);
         }
@@ -389,18 +340,42 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
     } else {
       block_scan_each<NT>(
           0, N, [&](int j) { return kept_pos(j); },
-          [&](int j, int rank) { sor[rank] = (uint16_t)j; }, warp_cnt);
+          [&](int j, int rank) { src_of_rank[rank] = (uint16_t)j; }, warp_cnt);
       for (int j = tid; j < N; j += NT)
         if (!kept_pos(j)) atomicMin(&first_evicted, j);
     }
     __syncthreads();
 
-    if (SPLIT) {  // the ranks are in the global buffer; the copy launch moves the rows
-      if (tid == 0) p.first_evicted[r * p.hkv + h] = first_evicted;
-      return;
-    }
     // 4. in-place, order-preserving copy of ranks [first_evicted, M)
-    copy_ranks<NT, kUnroll>(p, P, M, first_evicted, src_of_rank, row_of);
+    const int q0 = first_evicted;
+#pragma unroll 1
+    for (int base = q0; base < M; base += rows_per_pass * kUnroll) {
+      uint4 kr[kUnroll], vr[kUnroll];
+      int pr[kUnroll];
+      int64_t drow[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int q = base + u * rows_per_pass + my_row;
+        drow[u] = -1;
+        if (active && q < M) {
+          const int64_t srow = row_of(P + src_of_rank[q]);
+          drow[u] = row_of(P + q);
+          kr[u] = *reinterpret_cast<const uint4 *>(p.k_pool + srow * rb + my_vec * 16);
+          vr[u] = *reinterpret_cast<const uint4 *>(p.v_pool + srow * rb + my_vec * 16);
+          if (my_vec == 0) pr[u] = p.pos_map[srow];
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (drow[u] >= 0) {
+          *reinterpret_cast<uint4 *>(p.k_pool + drow[u] * rb + my_vec * 16) = kr[u];
+          *reinterpret_cast<uint4 *>(p.v_pool + drow[u] * rb + my_vec * 16) = vr[u];
+          if (my_vec == 0) p.pos_map[drow[u]] = pr[u];
+        }
+      }
+    }
+    if (tid == 0 && M > q0) atomicAdd(p.counters, (unsigned long long)(M - q0));
   } else {
     // 3'. holes (evicted candidates below M) and movers (kept at or past M),
     // each listed in candidate order: holes at src_of_rank[0..), movers at
@@ -443,50 +418,13 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
   }
 }
 
-// The copy half of a split round: ranks [first_evicted, M) of one segment
-// move as in the fused kernel, with the rank map staged from the global rank
-// buffer into shared memory first.
-template <int NT, int kUnroll>
-__global__ void __launch_bounds__(NT) compact_copy_kernel(SelectCompactParams p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint16_t *src_of_rank = reinterpret_cast<uint16_t *>(smem);  // [M] (entries below first_evicted unused)
-  const int tid = threadIdx.x;
-  const int h = blockIdx.x % p.hkv;
-  const int l = p.layer0 + (blockIdx.x / p.hkv) % p.nlayers;
-  const SegDesc sd = p.segs[blockIdx.x / (p.hkv * p.nlayers)];
-  const int r = sd.req, P = sd.P, M = sd.M;
-  const int32_t *bt = p.block_table + (int64_t)r * p.bt_stride;
-  const int64_t layer_page0 = (int64_t)l * p.num_pages;
-  auto row_of = [&](int s) -> int64_t {
-    return ((layer_page0 + bt[s >> 4]) * p.hkv + h) * kPage + (s & (kPage - 1));
-  };
-  const int q0 = p.first_evicted[r * p.hkv + h];
-  const uint16_t *rk = p.ranks + ((int64_t)r * p.hkv + h) * p.max_seq;
-  for (int q = q0 + tid; q < M; q += NT) src_of_rank[q] = rk[q];
-  __syncthreads();
-  copy_ranks<NT, kUnroll>(p, P, M, q0, src_of_rank, row_of);
-}
-
 template <int NT, int U, int MODE, int VAR>
 cudaError_t launch_one(const SelectCompactParams &p, int n_seg_req, int keys_cap, size_t smem,
                        cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(select_compact_kernel<NT, MODE, U, VAR, false>,
+  cudaError_t e = cudaFuncSetAttribute(select_compact_kernel<NT, MODE, U, VAR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  select_compact_kernel<NT, MODE, U, VAR, false><<<(unsigned)(n_seg_req * p.nlayers * p.hkv), NT, smem, s>>>(
-      p, keys_cap);
-  return cudaGetLastError();
-}
-
-template <int MODE, int VAR>
-cudaError_t launch_split_select(const SelectCompactParams &p, int n_seg_req, int keys_cap, cudaStream_t s) {
-  const size_t smem = (size_t)keys_cap * sizeof(uint32_t);  // keys only: the ranks go to global memory
-  cudaError_t e = cudaFuncSetAttribute(select_compact_kernel<256, MODE, 1, VAR, true>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  // 256 threads: with the Philox registers a 512-thread CTA would leave no
-  // room on its SM for a copy CTA of the previous layer
-  select_compact_kernel<256, MODE, 1, VAR, true><<<(unsigned)(n_seg_req * p.nlayers * p.hkv), 256, smem, s>>>(
+  select_compact_kernel<NT, MODE, U, VAR><<<(unsigned)(n_seg_req * p.layers * p.hkv), NT, smem, s>>>(
       p, keys_cap);
   return cudaGetLastError();
 }
@@ -516,34 +454,6 @@ cudaError_t launch_nt(const SelectCompactParams &p, int mode, int var, int n_seg
 }
 
 }  // namespace
-
-cudaError_t launch_select_ranks(const SelectCompactParams &p, int mode, int n_seg_req, int max_n, cudaStream_t s) {
-  if (n_seg_req <= 0) return cudaSuccess;
-  if (p.flags & kScHoleFill) return cudaErrorInvalidValue;
-  const bool by_pos = (p.flags & kScTieByPos) != 0;
-  const int keys_cap = (max_n + 7) & ~7;
-  switch (mode) {
-    case kModeRandom:
-      return by_pos ? launch_split_select<kModeRandom, kOrderedPosTie>(p, n_seg_req, keys_cap, s)
-                    : launch_split_select<kModeRandom, kOrderedSlotTie>(p, n_seg_req, keys_cap, s);
-    case kModeRandomShared:
-      return by_pos ? launch_split_select<kModeRandomShared, kOrderedPosTie>(p, n_seg_req, keys_cap, s)
-                    : launch_split_select<kModeRandomShared, kOrderedSlotTie>(p, n_seg_req, keys_cap, s);
-    default:
-      return by_pos ? launch_split_select<kModeScores, kOrderedPosTie>(p, n_seg_req, keys_cap, s)
-                    : launch_split_select<kModeScores, kOrderedSlotTie>(p, n_seg_req, keys_cap, s);
-  }
-}
-
-cudaError_t launch_compact_copy(const SelectCompactParams &p, int n_seg_req, int max_m, cudaStream_t s) {
-  if (n_seg_req <= 0) return cudaSuccess;
-  const size_t smem = (size_t)((max_m + 7) & ~7) * sizeof(uint16_t);
-  cudaError_t e = cudaFuncSetAttribute(compact_copy_kernel<256, KVC_SC_UNROLL_SMALL>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  compact_copy_kernel<256, KVC_SC_UNROLL_SMALL><<<(unsigned)(n_seg_req * p.nlayers * p.hkv), 256, smem, s>>>(p);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_select_compact(const SelectCompactParams &p, int mode, int n_seg_req,
                                   int max_n, int max_m, cudaStream_t s) {

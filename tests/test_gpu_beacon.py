@@ -334,17 +334,22 @@ def test_tcgen05_logit_far_above_running_max(B):
     print(B, out)
 
 
-@pytest.mark.parametrize("impl,B", [(1, 64), (2, 64), (2, 32), (2, 96), (2, 128), (2, 256)],
-                         ids=["simt-64", "tc-64", "tc-32", "tc-96", "tc-128", "tc-256"])
-def test_second_update_against_oracle(impl, B):
+@pytest.mark.parametrize("impl,B,W,Hq", [(1, 64, 64, 32), (2, 64, 64, 32), (2, 32, 64, 32), (2, 96, 64, 32),
+                                         (2, 128, 64, 32), (2, 256, 64, 32), (2, 64, 40, 32), (2, 64, 50, 16)],
+                         ids=["simt-64", "tc-64", "tc-32", "tc-96", "tc-128", "tc-256", "tc-64-160pts",
+                              "tc-64-G2-100pts"])
+def test_second_update_against_oracle(impl, B, W, Hq):
     """A later (non-initial) update: fp32 beacons with counts, new points.
     The oracle recomputes it from the GPU's beacons and counts before the
     update; assignments may differ only on near-ties within the kernels'
     error bound (fp32 rounding, plus 2^-18 sum|x_k c_k| per dot product for
-    the tensor-core kernel's two-term bf16 split of the beacons)."""
+    the tensor-core kernel's two-term bf16 split of the beacons).  The last
+    two cases leave the last 128-point tile partly filled (160 points; G = 2
+    with 100 points, a single partial tile)."""
     w = wl.beacon_serving(R=2, layers=2)
     w.num_beacons = B
-    w.query_window = max(64, B // 4)  # the first update needs at least B points
+    w.num_q_heads = Hq
+    w.query_window = max(W, B // (Hq // 8))  # the first update needs at least B points
     ctx = make_context(w, headroom=256)
     ctx.set_option(1, impl)
     gen = wl.Generator(w, "cuda")
@@ -354,7 +359,8 @@ def test_second_update_against_oracle(impl, B):
     st = ctx.state_tensors()
     c_before = st["beacons"].double().cpu().numpy()
     n_before = st["beacon_counts"].cpu().numpy().astype(np.int64)
-    R, Ly, H, d, G, W = 2, 2, 8, 128, 4, 64
+    R, Ly, H, d, G = 2, 2, 8, 128, Hq // 8
+    W = w.query_window
     q = gen.queries(R, W)
     k, v = gen.kv(R, W)
     ctx.append(np.arange(R, dtype=np.int32), k, v, q)
