@@ -16,7 +16,9 @@
 // most 2^-18 sum_k |x_k c_k| beyond fp32 rounding.  |c|^2 is the fp32 norm of
 // the fp32 beacon.  The per-beacon sums are a second tensor-core product of
 // one-hot assignment tiles with the same point tile (kernel comment below).
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
 
 #include "kvc_internal.h"
 #include "tc_ptx.cuh"
@@ -354,18 +356,26 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
 //               segment the assignment product of tile g+1 is issued before
 //               the sums of tile g, and a segment's last sums before the next
 //               segment's first assignment;
-//   warps 1-4   point warps: one point per thread.  Each thread copies its
-//               point of the tile D ahead with cp.async into one of NXS
-//               stages (128-byte-swizzled K-major layout; rows past the
-//               segment's points zero-filled), then takes the argmin over its
-//               TMEM lane of the assignment product, writes its one-hot entry
-//               and counts it;
+//   warps 1-4   point warps: one point per thread: the argmin over its TMEM
+//               lane of the assignment product, its one-hot entry and its
+//               count;
 //   warps 5-8   preparation: the next segment's beacons as bf16 hi/lo terms
 //               (swizzled, the B operand of the assignment) and their fp32
 //               squared norms;
 //   warps 9-12  running mean: one dimension per thread, over every beacon,
 //               (n c + sum) * (1 / (n + m)) with the reciprocal taken once
-//               per beacon.
+//               per beacon;
+//   warp 13     the point producer: one TMA box per 64-dimension half of a
+//               128-point tile into one of NXS stages (128-byte swizzle, the
+//               K-major A operand of the assignment).
+// The tiles walk the segment's query ring in physical slot order: tile t
+// holds slots [t S, t S + S) with S = 128 / G steps of G query heads, so a
+// tile is always one box and never wraps.  A point belongs to this update
+// when its slot's step lies in the update's window (the last n_steps steps,
+// starting at slot ring_start); the others (older queries, slots past W,
+// which read the next ring or the box's zero fill) are neither assigned nor
+// counted and leave a zero one-hot column, so their finite values add
+// nothing to the sums.  The ring is zeroed when the context is created.
 // The sums are D[dim][beacon] = X^T OH, with the point tile read as an
 // MN-major A operand (dimensions on M, its 64-dimension blocks 16 KB apart)
 // and the one-hot tile OH [beacon rows x point columns] as a K-major B
@@ -375,17 +385,9 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
 // (sums of neighbouring segments alternate).  The counts of three segments
 // rotate in shared memory so that the preparation never waits for a mean.
 // Every wait is bounded.
-constexpr int kPipeWarps = 13;
+constexpr int kPipeWarps = 14;
 constexpr int kPipeThreads = 32 * kPipeWarps;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // Every lane of the warp waits (bounded); the warp takes one decision.
@@ -406,7 +408,7 @@ __device__ __forceinline__ PipeSeg pipe_seg(const BeaconUpdateParams &p, int s) 
   const UpdateDesc ud = p.descs[s / (p.hkv * p.layers)];
   g.r = ud.req;
   g.n_pts = ud.n_steps * p.G;
-  g.T = (g.n_pts + 127) / 128;
+  g.T = (p.W * p.G + 127) / 128;  // tiles over every slot of the ring
   g.init = ud.init;
   g.ring_start = ud.ring_start;
   g.seg = ((int64_t)g.r * p.layers + g.l) * p.hkv + g.h;
@@ -421,9 +423,18 @@ __device__ __forceinline__ int64_t pipe_point(const BeaconUpdateParams &p, const
   return ((((int64_t)g.r * p.layers + g.l) * p.W + slot) * p.hq + (g.h * p.G + gq)) * 128;
 }
 
-template <int BM, int NXS, int NCB, int DA>
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+template <int BM, int NXS, int NCB>
 __global__ void __launch_bounds__(kPipeThreads, 1)
-    beacon_update_pipe_kernel(BeaconUpdateParams p, int n_segs) {
+    beacon_update_pipe_kernel(const __grid_constant__ CUtensorMap qmap, BeaconUpdateParams p, int n_segs) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_align<1024>(smem_raw);
   constexpr int D = 128;
@@ -438,7 +449,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   float *cn = reinterpret_cast<float *>(oh + 2 * kOHBytes);     // [NCB][BM] squared norms
   float *cpart = cn + NCB * BM;                                   // [2][4][BM] per-warp partial norms
   int32_t *cnt = reinterpret_cast<int32_t *>(cpart + 8 * BM);    // [3][BM] this update's counts
-  float *mfac = reinterpret_cast<float *>(cnt + 3 * BM);          // [2][2][BM] old count n, 1/(n+m) or 0
+  int32_t *nold = cnt + 3 * BM;                                   // [3][BM] counts before the update
+  float *mfac = reinterpret_cast<float *>(nold + 3 * BM);         // [2][2][BM] old count n, 1/(n+m) or 0
   uint64_t *bars = reinterpret_cast<uint64_t *>(mfac + 4 * BM);
   uint64_t *x_full = bars, *x_empty = x_full + NXS;
   uint64_t *prep_full = x_empty + NXS, *prep_empty = prep_full + NCB;
@@ -453,7 +465,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < NXS; ++i) {
-      mbar_init(&x_full[i], 128);  // the point threads' copies
+      mbar_init(&x_full[i], 1);  // the producer's expect_tx arrival; the box bytes complete it
       mbar_init(&x_empty[i], 1);
     }
     for (int i = 0; i < NCB; ++i) {
@@ -462,7 +474,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     }
     for (int i = 0; i < 3; ++i) {
       mbar_init(&cnt_full[i], 128);   // point warps: the segment's counts are complete
-      mbar_init(&cnt_empty[i], 128);  // mean warps: read and zeroed again
+      mbar_init(&cnt_empty[i], 128);  // mean warps: counts read and zeroed again
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -575,46 +587,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     int si = 0;
     bool ok = true, nan = false;
     uint32_t last_off0 = 0xffffffffu, last_off1 = 0xffffffffu;  // this point's entry in each one-hot tile
-    // load stream, DA tiles ahead of the argmins: this thread's point row of
-    // tile gl goes to stage gl % NXS
-    int ls = blockIdx.x, lt = 0;
-    bool lvalid = ls < n_segs;
-    PipeSeg lg = pipe_seg(p, lvalid ? ls : 0);
-    uint32_t gl = 0;
-    auto issue = [&]() -> bool {
-      const int st = gl % NXS;
-      if (!lanes_wait(&x_empty[st], ((gl / NXS) & 1) ^ 1, abort_flag, p.status)) return false;
-      uint8_t *dst = xs + st * kXBytes + row * 128;
-      const int pt = lt * 128 + row;
-      const bool valid = pt < lg.n_pts;
-      const __nv_bfloat16 *src = valid ? ring + pipe_point(p, lg, pt) : ring;
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        cp_async16(smem_u32(dst + (c >> 3) * 16384 + (((c & 7) ^ (row & 7)) << 4)), valid ? src + c * 8 : ring,
-                   valid ? 16u : 0u);
-      cp_async_commit();
-      ++gl;
-      if (++lt == lg.T) {
-        lt = 0;
-        ls += gridDim.x;
-        lvalid = ls < n_segs;
-        if (lvalid) lg = pipe_seg(p, ls);
-      }
-      return true;
-    };
-    for (int d = 0; d < DA && lvalid && ok; ++d) ok = issue();
-    // tile 0 is handed to the MMA here, tile g+1 at the start of iteration g,
-    // so that the assignment of tile g+1 runs during the argmin of tile g
-    uint32_t gs = 0;  // tiles handed to the MMA so far
-    auto hand = [&]() {
-      // tile gs has landed once at most gl - gs - 1 later groups are pending
-      if (DA >= 2 && gl - gs >= 2) cp_async_wait<1>();
-      else cp_async_wait<0>();
-      fence_proxy_async();
-      mbar_arrive(&x_full[gs % NXS]);
-      ++gs;
-    };
-    if (ok && gl > 0) hand();
+    const int S = 128 / p.G;                 // ring slots per tile
+    const int slot_in_tile = row / p.G, gq = row - (row / p.G) * p.G;
     for (int s = blockIdx.x; s < n_segs && ok; s += gridDim.x, ++si) {
       const PipeSeg g = pipe_seg(p, s);
       const int cb = si % NCB, kb3 = si % 3;
@@ -624,9 +598,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       const float *cnb = cn + cb * BM;
       int32_t *cntb = cnt + kb3 * BM;
       for (int t = 0; t < g.T; ++t, ++gi) {
-        if (gs < gl) hand();  // tile gi + 1
-        if (lvalid) ok = issue();
-        if (!ok) break;
+        // this row's slot; its step in the update's window, if it is in it
+        const int slot = t * S + slot_in_tile;
+        const int step = slot - g.ring_start + (slot < g.ring_start ? p.W : 0);
+        const bool valid = slot < p.W && step < g.n_pts / p.G;
+        const int pt = step * p.G + gq;
         const int ab = gi & 1;
         ok = lanes_wait(&acc_full[ab], (gi >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
@@ -639,7 +615,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float dist = fmaf(-2.f, v[i], cnb[c0 + i]);
-            nan |= (dist != dist);
+            nan |= valid && (dist != dist);
             if (dist < best) {
               best = dist;
               besti = c0 + i;
@@ -648,8 +624,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
         tmem_fence_before();
         mbar_arrive(&acc_empty[ab]);
-        const int pt = t * 128 + row;
-        const bool valid = pt < g.n_pts;
         if (valid) {
           if (p.assign_out) p.assign_out[g.seg * (int64_t)NP + pt] = besti;
           atomicAdd(&cntb[besti], 1);
@@ -673,7 +647,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       mbar_arrive(&cnt_full[kb3]);
       mbar_arrive(&prep_empty[cb]);
     }
-    cp_async_wait<0>();  // no copy outlives the CTA
     if (nan) atomicCAS(p.status, kDevOk, kDevNaN);
   } else if (warp < 9) {
     // --------------------------------------------------------- preparation
@@ -699,6 +672,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
       };
       load_batch(0);  // in flight while the buffer is still in use
+      // the old counts, for the running mean a segment or two later
+      const int n_old = (k < B && !g.init) ? p.counts[g.seg * B + k] : 0;
       ok = lanes_wait(&prep_empty[cb], ((si / NCB) & 1) ^ 1, abort_flag, p.status);
       if (!ok) break;
       for (int b0 = 0; b0 < B; b0 += 32) {
@@ -736,8 +711,41 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       ++ph;
       if (!ok) break;
       if (k < B) cn[cb * BM + k] = ((cp[k] + cp[BM + k]) + cp[2 * BM + k]) + cp[3 * BM + k];
+      // the count slot of this segment is free once the mean of segment si - 3 is done with it
+      ok = lanes_wait(&cnt_empty[si % 3], ((si / 3) & 1) ^ 1, abort_flag, p.status);
+      if (!ok) break;
+      if (k < B) nold[(si % 3) * BM + k] = n_old;
       mbar_arrive(&prep_full[cb]);
     }
+  } else if (warp == 13) {
+    // ------------------------------------------------------ point producer
+    if (lane == 0) {
+      uint32_t gl = 0;
+      bool ok = true;
+      const int S = 128 / p.G;
+      for (int s = blockIdx.x; s < n_segs && ok; s += gridDim.x) {
+        const PipeSeg g = pipe_seg(p, s);
+        const int z0 = (g.r * p.layers + g.l) * p.W;  // ring row of slot 0 of this (request, layer)
+        for (int t = 0; t < g.T; ++t, ++gl) {
+          const int st = gl % NXS;
+          ok = mbar_wait(&x_empty[st], ((gl / NXS) & 1) ^ 1, abort_flag, p.status);
+          if (!ok) break;
+          mbar_expect_tx(&x_full[st], kXBytes);
+          for (int kb = 0; kb < 2; ++kb)
+            tma_load_3d(smem_u32(xs + st * kXBytes + kb * 16384), &qmap, kb * 64, g.h * p.G, z0 + t * S,
+                        &x_full[st]);
+        }
+      }
+      if (*abort_flag && gl > 0) {
+        // let the boxes already issued land before the shared memory goes away
+        for (int i = 0; i < NXS; ++i) {
+          const uint32_t k = gl - 1 - i;
+          mbar_wait(&x_full[k % NXS], (k / NXS) & 1, abort_flag, p.status, false);
+          if (k == 0) break;
+        }
+      }
+    }
+    __syncwarp();
   } else {
     // -------------------------------------------------------- running mean
     const int q = warp & 3, k = q * 32 + lane;  // this thread's dimension = its TMEM lane
@@ -753,9 +761,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       int32_t *gcnt = p.counts + g.seg * B;
       __nv_bfloat16 *gs = reinterpret_cast<__nv_bfloat16 *>(p.beacons_s) + g.seg * B * D;
       float *nf = mfac + sb * 2 * BM, *inv = nf + BM;
-      // the old count and the first old values do not depend on this update's
-      // points: their loads fly while the sums are still being produced
-      const int n_old = (k < B && !g.init) ? gcnt[k] : 0;
+      // the first old values do not depend on this update's points: their
+      // loads fly while the sums are still being produced
       float onext[32];
       auto load_old = [&](int b0) {
         if (g.init) {
@@ -772,12 +779,18 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
            lanes_wait(&sum_full[sb], (si >> 1) & 1, abort_flag, p.status);
       if (!ok) break;
       tmem_fence_after();
-      // per beacon: n and 1/(n + m), or 0 when no point joined it (unchanged)
+      // per beacon: n and 1/(n + m), or 0 when no point joined it (unchanged);
+      // thread k is the only reader of count k, so it clears it at once and
+      // the count slot goes back to the point and preparation warps
+      int m = 0, n_old = 0;
       if (k < B) {
-        const int m = cntb[k];
+        m = cntb[k];
+        n_old = nold[kb3 * BM + k];
+        cntb[k] = 0;
         nf[k] = (float)n_old;
         inv[k] = m > 0 ? 1.f / (float)(n_old + m) : 0.f;
       }
+      mbar_arrive(&cnt_empty[kb3]);
       mbar_arrive(mean_sync);
       ok = lanes_wait(mean_sync, ph & 1, abort_flag, p.status);
       ++ph;
@@ -799,18 +812,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       }
       tmem_fence_before();
       mbar_arrive(&sum_empty[sb]);
-      // every thread has read all counts before they are zeroed
-      mbar_arrive(mean_sync);
-      ok = lanes_wait(mean_sync, ph & 1, abort_flag, p.status);
-      ++ph;
-      if (!ok) break;
       if (k < B) {
-        const int m = cntb[k];
         gcnt[k] = n_old + m;
         p.trig[g.seg * B + k] = (float)m / (float)g.n_pts;
-        cntb[k] = 0;
       }
-      mbar_arrive(&cnt_empty[kb3]);
     }
   }
   tmem_fence_before();
@@ -821,19 +826,48 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   }
 }
 
-template <int BM, int NXS, int NCB, int DA>
-cudaError_t launch_pipe(const BeaconUpdateParams &p, int n_segs, cudaStream_t s) {
+PFN_cuTensorMapEncodeTiled_v12000 tma_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// The query ring as (128 dimensions, Hq heads, R * layers * W slots) of bf16;
+// box (64 dimensions, G heads, 128 / G slots) = one 16 KB half of a point
+// tile in the 128-byte-swizzled K-major layout (row = slot * G + head).
+bool make_ring_map(CUtensorMap *m, const BeaconUpdateParams &p, int n_rows) {
+  auto fn = tma_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)p.hq, (cuuint64_t)n_rows};
+  cuuint64_t strides[2] = {256, (cuuint64_t)p.hq * 256};
+  cuuint32_t box[3] = {64, (cuuint32_t)p.G, (cuuint32_t)(128 / p.G)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint8_t *>(p.qring), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BM, int NXS, int NCB>
+cudaError_t launch_pipe(const BeaconUpdateParams &p, int n_segs, int n_rows, cudaStream_t s) {
+  CUtensorMap qmap;
+  if (!make_ring_map(&qmap, p, n_rows)) return cudaErrorInvalidValue;
   const size_t smem = 1024 + (size_t)NXS * 32768 + 2 * (size_t)NCB * BM * 256 + 2 * (size_t)BM * 256 +
-                      sizeof(float) * ((size_t)NCB * BM + 8 * BM + 4 * BM) + sizeof(int32_t) * 3 * (size_t)BM +
+                      sizeof(float) * ((size_t)NCB * BM + 8 * BM + 4 * BM) + sizeof(int32_t) * 6 * (size_t)BM +
                       8 * (2 * NXS + 2 * NCB + 6 + 12 + 3) + 16;  // barriers, TMEM slot, abort flag
-  cudaError_t e = cudaFuncSetAttribute(beacon_update_pipe_kernel<BM, NXS, NCB, DA>,
+  cudaError_t e = cudaFuncSetAttribute(beacon_update_pipe_kernel<BM, NXS, NCB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = n_segs < sms ? n_segs : sms;
-  beacon_update_pipe_kernel<BM, NXS, NCB, DA><<<grid, kPipeThreads, smem, s>>>(p, n_segs);
+  beacon_update_pipe_kernel<BM, NXS, NCB><<<grid, kPipeThreads, smem, s>>>(qmap, p, n_segs);
   return cudaGetLastError();
 }
 
@@ -850,8 +884,13 @@ cudaError_t launch_beacon_update_tc(const BeaconUpdateParams &p, int n_req, cuda
   // beacon), barrier/slot/flag; TMEM: assignment columns then 128 per half
   const size_t smem = 1024 + 32768 + (size_t)p.B * 512 + 32768 + (size_t)p.B * 4 * 6 + 64;
   const int n_segs = n_req * p.layers * p.hkv;
-  if (p.B <= 64) return launch_pipe<64, 3, 2, 2>(p, n_segs, s);
-  if (p.B <= 128) return launch_pipe<128, 2, 1, 1>(p, n_segs, s);
+  // the pipelined form: up to 128 beacons, G dividing 128 (a tile is whole
+  // ring slots), the ring addressable by the map's 32-bit slot coordinate
+  const int64_t ring_rows = (int64_t)p.n_ring * p.layers * p.W;
+  if (p.B <= 128 && 128 % p.G == 0 && ring_rows < (1ll << 31) && tma_encode_fn()) {
+    if (p.B <= 64) return launch_pipe<64, 3, 2>(p, n_segs, (int)ring_rows, s);
+    return launch_pipe<128, 2, 1>(p, n_segs, (int)ring_rows, s);
+  }
   const uint32_t cols = p.B <= 128 ? 256u : 512u;
   cudaError_t e = cudaFuncSetAttribute(beacon_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);

@@ -333,11 +333,12 @@ kvc_status kvc_create(const kvc_config *cfg, void *k_pool, void *v_pool, void *w
       return cleanup(e, "cudaEventCreate");
   for (auto &ev : c->ev)
     if ((e = cudaEventCreate(&ev)) != cudaSuccess) return cleanup(e, "cudaEventCreate");
-  // device state: block tables -1, lengths 0, position map -1, beacon counts 0
+  // device state: block tables -1, lengths 0, position map -1, query ring 0, beacon counts 0
   if ((e = cudaMemsetAsync(c->d_bt, 0xff, (size_t)R * c->maxp * 4, c->stream)) != cudaSuccess ||
       (e = cudaMemsetAsync(c->d_len, 0, (size_t)R * 4, c->stream)) != cudaSuccess ||
       (e = cudaMemsetAsync(c->d_prompt, 0, (size_t)R * 4, c->stream)) != cudaSuccess ||
       (e = cudaMemsetAsync(c->d_pos, 0xff, lay.qring - lay.pos, c->stream)) != cudaSuccess ||
+      (e = cudaMemsetAsync(c->d_qring, 0, lay.beacons - lay.qring, c->stream)) != cudaSuccess ||
       (e = cudaMemsetAsync(c->ws + lay.counts, 0, lay.scores - lay.counts, c->stream)) != cudaSuccess ||
       (e = cudaMemsetAsync(c->ws + lay.status, 0, lay.stage - lay.status, c->stream)) != cudaSuccess)
     return cleanup(e, "cudaMemsetAsync(workspace)");
@@ -526,6 +527,7 @@ kvc_status kvc_update_beacons(kvc_ctx *ctx, int32_t *assign_out, float *ms_out) 
   p.B = B;
   p.d = c.head_dim;
   p.dtype = c.dtype;
+  p.n_ring = c.num_requests;
   if (ms_out) KVC_CUDA(ctx, cudaEventRecord(ctx->ev[0], ctx->stream));
   const bool use_tc = ctx->update_impl == 2 ||
                       (ctx->update_impl == 0 && beacon_update_tc_supported(c.head_dim, B, c.dtype));

@@ -81,6 +81,7 @@ struct BeaconUpdateParams {
   const UpdateDesc *descs;
   int32_t *status;
   int32_t layers, hkv, hq, G, W, B, d, dtype;
+  int32_t n_ring;             // requests in the query ring (R)
 };
 
 // Beacon score over the paged keys of a segment.
