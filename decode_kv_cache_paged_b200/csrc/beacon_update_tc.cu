@@ -359,9 +359,9 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
 //   warps 1-4   point warps: one point per thread: the argmin over its TMEM
 //               lane of the assignment product, its one-hot entry and its
 //               count;
-//   warps 5-8   preparation: the next segment's beacons as bf16 hi/lo terms
-//               (swizzled, the B operand of the assignment) and their fp32
-//               squared norms;
+//   warps 5-8   preparation, one beacon per thread: the next segment's
+//               beacons as bf16 hi/lo terms (swizzled, the B operand of the
+//               assignment) and their fp32 squared norms;
 //   warps 9-12  running mean: one dimension per thread, over every beacon,
 //               (n c + sum) * (1 / (n + m)) with the reciprocal taken once
 //               per beacon;
@@ -382,8 +382,19 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
 // operand: a segment's sums take B TMEM columns, and the running mean reads
 // and writes each beacon row with one coalesced access per warp.
 // TMEM columns: two assignment buffers of BM, then two sums buffers of BM
-// (sums of neighbouring segments alternate).  The counts of three segments
-// rotate in shared memory so that the preparation never waits for a mean.
+// (sums of neighbouring segments alternate).  NOH one-hot tiles: two, or one
+// where shared memory is better spent on a third point stage.  The counts of
+// three segments rotate in shared memory so that the preparation never waits
+// for a mean.
+// More than 128 beacons: a cluster of two CTAs per segment (CL = 2), CTA r
+// holding beacons [128 r, 128 r + nb) with the layout above.  Both load the
+// same point tiles; each point thread takes the argmin over its CTA's
+// beacons and the two CTAs swap (distance, index) through distributed shared
+// memory (asynchronous stores completing on the peer's barriers, receipted
+// the same way), the lower half winning ties, so both hold the argmin over
+// every beacon.  Each CTA then writes the one-hot entries and counts of its
+// own beacons and runs their sums and means.  The pair prefetches its next
+// segment's beacons and point tiles into L2 while the current one runs.
 // Every wait is bounded.
 constexpr int kPipeWarps = 14;
 constexpr int kPipeThreads = 32 * kPipeWarps;
@@ -423,6 +434,73 @@ __device__ __forceinline__ int64_t pipe_point(const BeaconUpdateParams &p, const
   return ((((int64_t)g.r * p.layers + g.l) * p.W + slot) * p.hq + (g.h * p.G + gq)) * 128;
 }
 
+// Distributed shared memory between the two CTAs of a cluster.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+// Asynchronous stores into the peer CTA's shared memory, each completing as
+// transaction bytes on a barrier of the peer (whose complete-tx releases the
+// bytes at cluster scope): no fence on the sending side.
+__device__ __forceinline__ void st_async_v2(uint32_t caddr, float a, int32_t b, uint32_t cbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(caddr),
+               "r"(__float_as_int(a)), "r"(b), "r"(cbar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_b32(uint32_t caddr, int32_t a, uint32_t cbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(caddr), "r"(a),
+               "r"(cbar)
+               : "memory");
+}
+// Bounded wait whose acquire covers stores made by the peer CTA.
+__device__ __forceinline__ bool mbar_wait_cl(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             int32_t *status, bool honor_abort = true) {
+  auto try_once = [&]() {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+        : "memory");
+    return ok != 0;
+  };
+  if (try_once()) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (try_once()) return true;
+    if (honor_abort && *abort_flag) return false;
+    if (global_ns() - t0 > kWaitNs) {
+      atomicCAS(status, kDevOk, kDevTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// L2 prefetches: `bytes` contiguous bytes (16-byte aligned, a multiple of
+// 16), and one box of a tensor map.  Neither writes shared memory.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void prefetch_box_3d(const CUtensorMap *map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z,
                                             uint64_t *bar) {
   asm volatile(
@@ -432,7 +510,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
-template <int BM, int NXS, int NCB>
+template <int BM, int NXS, int NCB, int NOH, int CL>
 __global__ void __launch_bounds__(kPipeThreads, 1)
     beacon_update_pipe_kernel(const __grid_constant__ CUtensorMap qmap, BeaconUpdateParams p, int n_segs) {
   extern __shared__ uint8_t smem_raw[];
@@ -441,14 +519,22 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   constexpr uint32_t kXBytes = 32768;    // 128 points x 128 bf16
   constexpr uint32_t kCBytes = BM * 256;  // one term of one beacon buffer: [2 K-blocks][B rows][128 B]
   constexpr uint32_t kOHBytes = BM * 256; // one one-hot tile: [2 point blocks][B rows][128 B]
-  const int B = p.B;
+  // this CTA's beacons: [b_lo, b_lo + B) of the segment's Bg
+  const int Bg = p.B;
+  const uint32_t rank = CL > 1 ? cluster_rank() : 0u;
+  const int b_lo = (int)rank * 128;
+  const int B = CL > 1 ? (rank ? Bg - 128 : 128) : Bg;
+  const int seg0 = blockIdx.x / CL, seg_step = gridDim.x / CL;
   uint8_t *xs = smem;
   uint8_t *chi = xs + NXS * kXBytes;
   uint8_t *clo = chi + NCB * kCBytes;
   uint8_t *oh = clo + NCB * kCBytes;
-  float *cn = reinterpret_cast<float *>(oh + 2 * kOHBytes);     // [NCB][BM] squared norms
-  float *cpart = cn + NCB * BM;                                   // [2][4][BM] per-warp partial norms
-  int32_t *cnt = reinterpret_cast<int32_t *>(cpart + 8 * BM);    // [3][BM] this update's counts
+  // squared norms: a ring of NCB + 2, so that the preparation of segment
+  // si + NCB (which starts once the MMA has read segment si's terms) never
+  // overwrites the norms of a segment the point warps may still scan
+  constexpr int NCN = NCB + 2;
+  float *cn = reinterpret_cast<float *>(oh + NOH * kOHBytes);   // [NCN][BM] squared norms
+  int32_t *cnt = reinterpret_cast<int32_t *>(cn + NCN * BM);     // [3][BM] this update's counts
   int32_t *nold = cnt + 3 * BM;                                   // [3][BM] counts before the update
   float *mfac = reinterpret_cast<float *>(nold + 3 * BM);         // [2][2][BM] old count n, 1/(n+m) or 0
   uint64_t *bars = reinterpret_cast<uint64_t *>(mfac + 4 * BM);
@@ -458,8 +544,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   uint64_t *acc_full = cnt_empty + 3, *acc_empty = acc_full + 2;
   uint64_t *oh_full = acc_empty + 2, *oh_empty = oh_full + 2;
   uint64_t *sum_full = oh_empty + 2, *sum_empty = sum_full + 2;
-  uint64_t *prep_sync = sum_empty + 2, *mean_sync = prep_sync + 1, *mma_done = mean_sync + 1;
-  uint32_t *tslot = reinterpret_cast<uint32_t *>(mma_done + 1);
+  uint64_t *mean_sync = sum_empty + 2, *mma_done = mean_sync + 1;
+  uint64_t *xch_full = mma_done + 1, *xch_empty = xch_full + 2;  // the argmin swap (CL = 2)
+  float2 *xch = reinterpret_cast<float2 *>(xch_empty + 2);          // [2][128] the peer's (distance, index)
+  int32_t *ack = reinterpret_cast<int32_t *>(xch + (CL > 1 ? 256 : 0));  // [2][128] the peer's receipts
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(ack + (CL > 1 ? 256 : 0));
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -470,7 +559,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     }
     for (int i = 0; i < NCB; ++i) {
       mbar_init(&prep_full[i], 128);
-      mbar_init(&prep_empty[i], 1 + 128);  // MMA commit, point warps
+      mbar_init(&prep_empty[i], 1);  // MMA commit after the segment's last assignment
     }
     for (int i = 0; i < 3; ++i) {
       mbar_init(&cnt_full[i], 128);   // point warps: the segment's counts are complete
@@ -484,15 +573,25 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       mbar_init(&sum_full[i], 1);
       mbar_init(&sum_empty[i], 128);
     }
-    mbar_init(prep_sync, 128);
     mbar_init(mean_sync, 128);
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      // completed by the peer's stores: its 128 argmins in xch (8 bytes each),
+      // its 128 receipts for ours (4 bytes each); each phase is armed by this
+      // CTA's point thread 0 one phase ahead, the first ones here
+      mbar_init(&xch_full[i], 1);
+      mbar_init(&xch_empty[i], 1);
+      if (CL > 1) {
+        mbar_expect_tx(&xch_full[i], 128 * 8);
+        mbar_expect_tx(&xch_empty[i], 128 * 4);
+      }
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // the one-hot tiles start at zero (each point clears its own entry later),
   // and so do the count buffers (the mean warps zero each after reading it)
-  for (int i = tid; i < (int)(2 * kOHBytes / 16); i += kPipeThreads)
+  for (int i = tid; i < (int)(NOH * kOHBytes / 16); i += kPipeThreads)
     reinterpret_cast<uint4 *>(oh)[i] = make_uint4(0, 0, 0, 0);
   for (int i = tid; i < 3 * BM; i += kPipeThreads) cnt[i] = 0;
   fence_proxy_async();
@@ -503,6 +602,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   }
   tmem_fence_before();
   __syncthreads();
+  if constexpr (CL > 1) cluster_sync_all();  // the peer's barriers are initialised
   tmem_fence_after();
   const uint32_t tmem_base = *tslot;
   const __nv_bfloat16 *ring = reinterpret_cast<const __nv_bfloat16 *>(p.qring);
@@ -534,11 +634,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       };
       auto sums = [&](uint32_t gi, int si, int t, int T) {
         const int sb = si & 1;
-        ok = ok && mbar_wait(&oh_full[gi & 1], (gi >> 1) & 1, abort_flag, p.status);
+        ok = ok && mbar_wait(&oh_full[gi % NOH], (gi / NOH) & 1, abort_flag, p.status);
         if (t == 0) ok = ok && mbar_wait(&sum_empty[sb], ((si >> 1) & 1) ^ 1, abort_flag, p.status);
         if (!ok) return;
         tmem_fence_after();
-        const uint32_t xa = smem_u32(xs + (gi % NXS) * kXBytes), oa = smem_u32(oh + (gi & 1) * kOHBytes);
+        const uint32_t xa = smem_u32(xs + (gi % NXS) * kXBytes), oa = smem_u32(oh + (gi % NOH) * kOHBytes);
         for (int ks = 0; ks < 8; ++ks) {
           // X^T: 16 points from point group ks, 64-dimension blocks 16 KB apart (LBO), 8-point groups 1 KB
           // apart (SBO)
@@ -548,7 +648,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           umma(tmem_base + 2 * BM + sb * BM, a, bd, idesc_sum, (t > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit(&x_empty[gi % NXS]);
-        umma_commit(&oh_empty[gi & 1]);
+        umma_commit(&oh_empty[gi % NOH]);
         if (t == T - 1) umma_commit(&sum_full[sb]);
       };
       // tile stream; the assignment runs one tile ahead of the sums
@@ -560,7 +660,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       // within a segment; at a segment boundary the last sums go first, so
       // that the running mean of a segment never waits for the next
       // segment's beacon preparation
-      for (int s = blockIdx.x; s < n_segs && ok; s += gridDim.x, ++si) {
+      for (int s = seg0; s < n_segs && ok; s += seg_step, ++si) {
         const PipeSeg g = pipe_seg(p, s);
         for (int t = 0; t < g.T && ok; ++t, ++gi) {
           if (have_prev && t == 0) sums(pg, ps, pt, pT);
@@ -589,13 +689,20 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     uint32_t last_off0 = 0xffffffffu, last_off1 = 0xffffffffu;  // this point's entry in each one-hot tile
     const int S = 128 / p.G;                 // ring slots per tile
     const int slot_in_tile = row / p.G, gq = row - (row / p.G) * p.G;
-    for (int s = blockIdx.x; s < n_segs && ok; s += gridDim.x, ++si) {
+    uint32_t peer_xch = 0, peer_ack = 0, peer_full = 0, peer_empty = 0;
+    if constexpr (CL > 1) {
+      peer_xch = map_peer(smem_u32(xch), rank ^ 1u);
+      peer_ack = map_peer(smem_u32(ack), rank ^ 1u);
+      peer_full = map_peer(smem_u32(xch_full), rank ^ 1u);
+      peer_empty = map_peer(smem_u32(xch_empty), rank ^ 1u);
+    }
+    for (int s = seg0; s < n_segs && ok; s += seg_step, ++si) {
       const PipeSeg g = pipe_seg(p, s);
       const int cb = si % NCB, kb3 = si % 3;
       ok = lanes_wait(&prep_full[cb], (si / NCB) & 1, abort_flag, p.status) &&
            lanes_wait(&cnt_empty[kb3], ((si / 3) & 1) ^ 1, abort_flag, p.status);
       if (!ok) break;
-      const float *cnb = cn + cb * BM;
+      const float *cnb = cn + (si % NCN) * BM;
       int32_t *cntb = cnt + kb3 * BM;
       for (int t = 0; t < g.T; ++t, ++gi) {
         // this row's slot; its step in the update's window, if it is in it
@@ -607,8 +714,16 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         ok = lanes_wait(&acc_full[ab], (gi >> 1) & 1, abort_flag, p.status);
         if (!ok) break;
         tmem_fence_after();
-        float best = __int_as_float(0x7f800000);
-        int besti = 0;
+        // four interleaved chains (column i in chain i % 4), each keeping its
+        // first minimum; merged by value, then by the lower index, which is
+        // the first minimum of one pass over every column
+        float bst[4];
+        int bix[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          bst[j] = __int_as_float(0x7f800000);
+          bix[j] = 0;
+        }
         for (int c0 = 0; c0 < B; c0 += 32) {
           float v[32];
           tmem_ld32(tmem_base + lane_addr + ab * BM + c0, v);
@@ -616,105 +731,155 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           for (int i = 0; i < 32; ++i) {
             const float dist = fmaf(-2.f, v[i], cnb[c0 + i]);
             nan |= valid && (dist != dist);
-            if (dist < best) {
-              best = dist;
-              besti = c0 + i;
+            if (dist < bst[i & 3]) {
+              bst[i & 3] = dist;
+              bix[i & 3] = c0 + i;
             }
           }
         }
+        float best = bst[0];
+        int besti = bix[0];
+#pragma unroll
+        for (int j = 1; j < 4; ++j)
+          if (bst[j] < best || (bst[j] == best && bix[j] < besti)) {
+            best = bst[j];
+            besti = bix[j];
+          }
         tmem_fence_before();
         mbar_arrive(&acc_empty[ab]);
-        if (valid) {
-          if (p.assign_out) p.assign_out[g.seg * (int64_t)NP + pt] = besti;
-          atomicAdd(&cntb[besti], 1);
+        int fin = besti + b_lo;  // the argmin over the segment's beacons
+        if constexpr (CL > 1) {
+          // swap with the peer: wait until it has receipted what this thread
+          // put in its slot two tiles ago, send, then read the peer's entry
+          // here and receipt it (the receipt carries the value read)
+          ok = __all_sync(0xffffffffu, mbar_wait_cl(&xch_empty[ab], ((gi >> 1) & 1) ^ 1, abort_flag, p.status));
+          if (!ok) break;
+          if (row == 0 && gi >= 2) mbar_expect_tx(&xch_empty[ab], 128 * 4);  // receipts for this tile's entries
+          st_async_v2(peer_xch + (ab * 128 + row) * 8, best, fin, peer_full + ab * 8);
+          ok = __all_sync(0xffffffffu, mbar_wait_cl(&xch_full[ab], (gi >> 1) & 1, abort_flag, p.status));
+          if (!ok) break;
+          const float2 o = xch[ab * 128 + row];
+          if (row == 0) mbar_expect_tx(&xch_full[ab], 128 * 8);  // the peer's argmins of tile gi + 2
+          st_async_b32(peer_ack + (ab * 128 + row) * 4, __float_as_int(o.y), peer_empty + ab * 8);
+          // lower beacon indices win ties, as in one pass over every beacon
+          if (rank == 0 ? (o.x < best) : !(best < o.x)) fin = __float_as_int(o.y);
         }
-        ok = lanes_wait(&oh_empty[ab], ((gi >> 1) & 1) ^ 1, abort_flag, p.status);
+        const bool mine = valid && fin >= b_lo && fin < b_lo + B;
+        if (valid) {
+          if (p.assign_out && rank == 0) p.assign_out[g.seg * (int64_t)NP + pt] = fin;
+          if (mine) atomicAdd(&cntb[fin - b_lo], 1);
+        }
+        const int ob = gi % NOH;
+        ok = lanes_wait(&oh_empty[ob], ((gi / NOH) & 1) ^ 1, abort_flag, p.status);
         if (!ok) break;
-        uint8_t *ohb = oh + ab * kOHBytes;
-        const uint32_t prev = ab ? last_off1 : last_off0;
+        uint8_t *ohb = oh + ob * kOHBytes;
+        const uint32_t prev = ob ? last_off1 : last_off0;
         if (prev != 0xffffffffu) *reinterpret_cast<uint16_t *>(ohb + prev) = 0;
         uint32_t off = 0xffffffffu;
-        if (valid) {
-          off = (uint32_t)(row >> 6) * (uint32_t)B * 128u + sw128_off(besti, row & 63);
+        if (mine) {
+          off = (uint32_t)(row >> 6) * (uint32_t)B * 128u + sw128_off(fin - b_lo, row & 63);
           *reinterpret_cast<uint16_t *>(ohb + off) = 0x3F80;  // bf16 1.0
         }
-        if (ab) last_off1 = off;
+        if (ob) last_off1 = off;
         else last_off0 = off;
         fence_proxy_async();
-        mbar_arrive(&oh_full[ab]);
+        mbar_arrive(&oh_full[ob]);
       }
       if (!ok) break;
       mbar_arrive(&cnt_full[kb3]);
-      mbar_arrive(&prep_empty[cb]);
+    }
+    if constexpr (CL > 1) {
+      // the peer's receipts for the last two tiles land before this CTA may
+      // leave (bounded by time alone, also after an abort)
+      for (uint32_t gt = gi >= 2 ? gi - 2 : 0; gt < gi; ++gt)
+        mbar_wait_cl(&xch_empty[gt & 1], (((gt + 2) >> 1) & 1) ^ 1, abort_flag, p.status, false);
     }
     if (nan) atomicCAS(p.status, kDevOk, kDevNaN);
   } else if (warp < 9) {
     // --------------------------------------------------------- preparation
-    const int w6 = warp - 5, k = w6 * 32 + lane;  // this thread's dimension
+    // thread b: beacon b of this CTA's share, its 128 dimensions in four
+    // quarters of 32 (the next quarter's loads in flight): bf16 hi/lo terms
+    // written as 16-byte chunks of the swizzled layout, and the squared norm
+    // as one running fp32 sum over the dimensions
+    const int b = (warp - 5) * 32 + lane;
     int si = 0;
-    uint32_t ph = 0;
     bool ok = true;
-    for (int s = blockIdx.x; s < n_segs && ok; s += gridDim.x, ++si) {
+    for (int s = seg0; s < n_segs && ok; s += seg_step, ++si) {
       const PipeSeg g = pipe_seg(p, s);
       const int cb = si % NCB;
-      const float *gbeac = p.beacons + g.seg * B * D;
-      float *cp = cpart + (si & 1) * 4 * BM;
+      const bool have = b < B;
       uint8_t *hb = chi + cb * kCBytes, *lb = clo + cb * kCBytes;
-      float cnext[32];
-      auto load_batch = [&](int b0) {
+      const float *frow = p.beacons + (g.seg * Bg + b_lo + b) * D;
+      const __nv_bfloat16 *irow =
+          ring + pipe_point(p, g, (int)(((int64_t)(b_lo + (have ? b : 0)) * g.n_pts) / Bg));
+      float4 qn[8];
+      auto load_q = [&](int kq) {
+        if (!have) return;
         if (g.init) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(irow + kq * 32);
 #pragma unroll
-          for (int u = 0; u < 32; ++u)
-            cnext[u] = __bfloat162float(ring[pipe_point(p, g, (int)(((int64_t)(b0 + u) * g.n_pts) / B)) + k]);
+          for (int j = 0; j < 4; ++j) {
+            const uint4 w = src[j];  // 8 bf16, the lower element in the lower half
+            qn[2 * j] = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                                    __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+            qn[2 * j + 1] = make_float4(__uint_as_float(w.z << 16), __uint_as_float(w.z & 0xffff0000u),
+                                        __uint_as_float(w.w << 16), __uint_as_float(w.w & 0xffff0000u));
+          }
         } else {
+          const float4 *src = reinterpret_cast<const float4 *>(frow + kq * 32);
 #pragma unroll
-          for (int u = 0; u < 32; ++u) cnext[u] = gbeac[(b0 + u) * D + k];
+          for (int j = 0; j < 8; ++j) qn[j] = src[j];
         }
       };
-      load_batch(0);  // in flight while the buffer is still in use
-      // the old counts, for the running mean a segment or two later
-      const int n_old = (k < B && !g.init) ? p.counts[g.seg * B + k] : 0;
+      load_q(0);  // in flight while the buffer is still in use
+      // the pair form: this CTA's beacons of its next segment into L2
+      if (CL > 1 && b == 0 && s + seg_step < n_segs) {
+        const PipeSeg gn = pipe_seg(p, s + seg_step);
+        prefetch_l2(p.beacons + (gn.seg * Bg + b_lo) * D, (uint32_t)(B * D * sizeof(float)));
+      }
+      // the old count, for the running mean a segment or two later
+      const int n_old = (have && !g.init) ? p.counts[g.seg * Bg + b_lo + b] : 0;
       ok = lanes_wait(&prep_empty[cb], ((si / NCB) & 1) ^ 1, abort_flag, p.status);
       if (!ok) break;
-      for (int b0 = 0; b0 < B; b0 += 32) {
+      float nrm = 0.f;
+#pragma unroll 1
+      for (int kq = 0; kq < 4; ++kq) {
         float c[32];
 #pragma unroll
-        for (int u = 0; u < 32; ++u) c[u] = cnext[u];
-        if (b0 + 32 < B) load_batch(b0 + 32);
-        const uint32_t kbo = (uint32_t)(k >> 6) * (uint32_t)B * 128u;
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const __nv_bfloat16 hi = __float2bfloat16_rn(c[u]);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(c[u] - __bfloat162float(hi));
-          const uint32_t off = kbo + sw128_off(b0 + u, k & 63);
-          *reinterpret_cast<__nv_bfloat16 *>(hb + off) = hi;
-          *reinterpret_cast<__nv_bfloat16 *>(lb + off) = lo;
-          c[u] = c[u] * c[u];
+        for (int j = 0; j < 8; ++j) {
+          c[4 * j] = qn[j].x;
+          c[4 * j + 1] = qn[j].y;
+          c[4 * j + 2] = qn[j].z;
+          c[4 * j + 3] = qn[j].w;
         }
-        // butterfly reduce-scatter of the 32 squares over the warp's 32
-        // dimensions: lane j ends with beacon b0 + j's partial norm
+        if (kq < 3) load_q(kq + 1);
+        if (!have) continue;
 #pragma unroll
-        for (int w = 16; w >= 1; w >>= 1) {
-          const bool up = (lane & w) != 0;
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t h[4], l[4];
 #pragma unroll
-          for (int i = 0; i < w; ++i) {
-            const float send = up ? c[i] : c[i + w];
-            const float keep = up ? c[i + w] : c[i];
-            c[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = c[ch * 8 + 2 * e], x1 = c[ch * 8 + 2 * e + 1];
+            const __nv_bfloat162 hh = __floats2bfloat162_rn(x0, x1);
+            const float2 hf = __bfloat1622float2(hh);
+            const __nv_bfloat162 ll = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+            h[e] = *reinterpret_cast<const uint32_t *>(&hh);
+            l[e] = *reinterpret_cast<const uint32_t *>(&ll);
           }
+          const int kk = kq * 32 + ch * 8;  // the chunk's first dimension
+          const uint32_t off = (uint32_t)(kk >> 6) * (uint32_t)B * 128u + sw128_off(b, kk & 63);
+          *reinterpret_cast<uint4 *>(hb + off) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4 *>(lb + off) = make_uint4(l[0], l[1], l[2], l[3]);
         }
-        cp[w6 * BM + b0 + lane] = c[0];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) nrm = fmaf(c[i], c[i], nrm);
       }
+      if (have) cn[(si % NCN) * BM + b] = nrm;
       fence_proxy_async();  // the beacon terms, for the MMA
-      mbar_arrive(prep_sync);
-      ok = lanes_wait(prep_sync, ph & 1, abort_flag, p.status);
-      ++ph;
-      if (!ok) break;
-      if (k < B) cn[cb * BM + k] = ((cp[k] + cp[BM + k]) + cp[2 * BM + k]) + cp[3 * BM + k];
       // the count slot of this segment is free once the mean of segment si - 3 is done with it
       ok = lanes_wait(&cnt_empty[si % 3], ((si / 3) & 1) ^ 1, abort_flag, p.status);
       if (!ok) break;
-      if (k < B) nold[(si % 3) * BM + k] = n_old;
+      if (have) nold[(si % 3) * BM + b] = n_old;
       mbar_arrive(&prep_full[cb]);
     }
   } else if (warp == 13) {
@@ -723,9 +888,16 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       uint32_t gl = 0;
       bool ok = true;
       const int S = 128 / p.G;
-      for (int s = blockIdx.x; s < n_segs && ok; s += gridDim.x) {
+      for (int s = seg0; s < n_segs && ok; s += seg_step) {
         const PipeSeg g = pipe_seg(p, s);
         const int z0 = (g.r * p.layers + g.l) * p.W;  // ring row of slot 0 of this (request, layer)
+        // the pair form: the next segment's point tiles into L2 (one CTA)
+        if (CL > 1 && rank == 0 && s + seg_step < n_segs) {
+          const PipeSeg gn = pipe_seg(p, s + seg_step);
+          const int zn = (gn.r * p.layers + gn.l) * p.W;
+          for (int t = 0; t < gn.T; ++t)
+            for (int kb = 0; kb < 2; ++kb) prefetch_box_3d(&qmap, kb * 64, gn.h * p.G, zn + t * S);
+        }
         for (int t = 0; t < g.T; ++t, ++gl) {
           const int st = gl % NXS;
           ok = mbar_wait(&x_empty[st], ((gl / NXS) & 1) ^ 1, abort_flag, p.status);
@@ -753,13 +925,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     int si = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int s = blockIdx.x; s < n_segs && ok; s += gridDim.x, ++si) {
+    for (int s = seg0; s < n_segs && ok; s += seg_step, ++si) {
       const PipeSeg g = pipe_seg(p, s);
       const int kb3 = si % 3, sb = si & 1;
       int32_t *cntb = cnt + kb3 * BM;
-      float *gbeac = p.beacons + g.seg * B * D;
-      int32_t *gcnt = p.counts + g.seg * B;
-      __nv_bfloat16 *gs = reinterpret_cast<__nv_bfloat16 *>(p.beacons_s) + g.seg * B * D;
+      float *gbeac = p.beacons + (g.seg * Bg + b_lo) * D;
+      int32_t *gcnt = p.counts + g.seg * Bg + b_lo;
+      __nv_bfloat16 *gs = reinterpret_cast<__nv_bfloat16 *>(p.beacons_s) + (g.seg * Bg + b_lo) * D;
       float *nf = mfac + sb * 2 * BM, *inv = nf + BM;
       // the first old values do not depend on this update's points: their
       // loads fly while the sums are still being produced
@@ -768,7 +940,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         if (g.init) {
 #pragma unroll
           for (int u = 0; u < 32; ++u)
-            onext[u] = __bfloat162float(ring[pipe_point(p, g, (int)(((int64_t)(b0 + u) * g.n_pts) / B)) + k]);
+            onext[u] =
+                __bfloat162float(ring[pipe_point(p, g, (int)(((int64_t)(b_lo + b0 + u) * g.n_pts) / Bg)) + k]);
         } else {
 #pragma unroll
           for (int u = 0; u < 32; ++u) onext[u] = gbeac[(b0 + u) * D + k];
@@ -814,12 +987,14 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       mbar_arrive(&sum_empty[sb]);
       if (k < B) {
         gcnt[k] = n_old + m;
-        p.trig[g.seg * B + k] = (float)m / (float)g.n_pts;
+        p.trig[g.seg * Bg + b_lo + k] = (float)m / (float)g.n_pts;
       }
     }
   }
   tmem_fence_before();
   __syncthreads();
+  // neither CTA leaves while the other may still write into its shared memory
+  if constexpr (CL > 1) cluster_sync_all();
   if (warp == 0) {
     tmem_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(4 * BM));
@@ -853,22 +1028,45 @@ bool make_ring_map(CUtensorMap *m, const BeaconUpdateParams &p, int n_rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BM, int NXS, int NCB>
+template <int BM, int NXS, int NCB, int NOH, int CL>
 cudaError_t launch_pipe(const BeaconUpdateParams &p, int n_segs, int n_rows, cudaStream_t s) {
   CUtensorMap qmap;
   if (!make_ring_map(&qmap, p, n_rows)) return cudaErrorInvalidValue;
-  const size_t smem = 1024 + (size_t)NXS * 32768 + 2 * (size_t)NCB * BM * 256 + 2 * (size_t)BM * 256 +
-                      sizeof(float) * ((size_t)NCB * BM + 8 * BM + 4 * BM) + sizeof(int32_t) * 6 * (size_t)BM +
-                      8 * (2 * NXS + 2 * NCB + 6 + 12 + 3) + 16;  // barriers, TMEM slot, abort flag
-  cudaError_t e = cudaFuncSetAttribute(beacon_update_pipe_kernel<BM, NXS, NCB>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = 1024 + (size_t)NXS * 32768 + 2 * (size_t)NCB * BM * 256 + (size_t)NOH * BM * 256 +
+                      sizeof(float) * ((size_t)(NCB + 2) * BM + 4 * BM) + sizeof(int32_t) * 6 * (size_t)BM +
+                      8 * (2 * NXS + 2 * NCB + 6 + 12 + 2 + 4) + (CL > 1 ? 256 * 12 : 0) +
+                      16;  // barriers, swap slots, TMEM slot, abort flag
+  auto kernel = beacon_update_pipe_kernel<BM, NXS, NCB, NOH, CL>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = n_segs < sms ? n_segs : sms;
-  beacon_update_pipe_kernel<BM, NXS, NCB><<<grid, kPipeThreads, smem, s>>>(qmap, p, n_segs);
-  return cudaGetLastError();
+  if (CL == 1) {
+    const int grid = n_segs < sms ? n_segs : sms;
+    kernel<<<grid, kPipeThreads, smem, s>>>(qmap, p, n_segs);
+    return cudaGetLastError();
+  }
+  // one cluster per segment at a time, as many clusters as fit at once
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kPipeThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3((unsigned)(CL * (sms / CL)));
+  int clusters = 0;
+  e = cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg);
+  if (e != cudaSuccess) return e;
+  if (clusters <= 0) return cudaErrorNotSupported;
+  if (clusters > n_segs) clusters = n_segs;
+  cfg.gridDim = dim3((unsigned)(CL * clusters));
+  return cudaLaunchKernelEx(&cfg, kernel, qmap, p, n_segs);
 }
 
 }  // namespace
@@ -884,12 +1082,18 @@ cudaError_t launch_beacon_update_tc(const BeaconUpdateParams &p, int n_req, cuda
   // beacon), barrier/slot/flag; TMEM: assignment columns then 128 per half
   const size_t smem = 1024 + 32768 + (size_t)p.B * 512 + 32768 + (size_t)p.B * 4 * 6 + 64;
   const int n_segs = n_req * p.layers * p.hkv;
-  // the pipelined form: up to 128 beacons, G dividing 128 (a tile is whole
-  // ring slots), the ring addressable by the map's 32-bit slot coordinate
+  // the pipelined form: G dividing 128 (a tile is whole ring slots), the ring
+  // addressable by the map's 32-bit slot coordinate
   const int64_t ring_rows = (int64_t)p.n_ring * p.layers * p.W;
   if (p.B <= 128 && 128 % p.G == 0 && ring_rows < (1ll << 31) && tma_encode_fn()) {
-    if (p.B <= 64) return launch_pipe<64, 3, 2>(p, n_segs, (int)ring_rows, s);
-    return launch_pipe<128, 2, 1>(p, n_segs, (int)ring_rows, s);
+    if (p.B <= 64) return launch_pipe<64, 3, 2, 2, 1>(p, n_segs, (int)ring_rows, s);
+    return launch_pipe<128, 2, 1, 2, 1>(p, n_segs, (int)ring_rows, s);
+  }
+  if (128 % p.G == 0 && ring_rows < (1ll << 31) && tma_encode_fn()) {
+    // more than 128 beacons: a CTA pair per segment, 128 beacons in the first;
+    // one one-hot buffer buys a third point stage
+    const cudaError_t e = launch_pipe<128, 3, 1, 1, 2>(p, n_segs, (int)ring_rows, s);
+    if (e != cudaErrorNotSupported) return e;
   }
   const uint32_t cols = p.B <= 128 ? 256u : 512u;
   cudaError_t e = cudaFuncSetAttribute(beacon_update_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
