@@ -60,6 +60,7 @@ def parse():
     ap.add_argument("--selector", default=None, help="override the workload's selector")
     ap.add_argument("--requests", type=int, default=None)
     ap.add_argument("--layers", type=int, default=None)
+    ap.add_argument("--beacons", type=int, default=None, help="override the workload's beacon count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-cpu-pool", action="store_true",
                     help="skip timing the oracle over all host cores (one spawned process per core)")
@@ -111,6 +112,8 @@ def make_workload(args):
         kw["num_requests"] = args.requests
     if args.layers:
         kw["num_layers"] = args.layers
+    if getattr(args, "beacons", None):
+        kw["num_beacons"] = args.beacons
     if kw:
         w = wl.scaled(w, **kw)
     sel = args.selector or w.selectors[0]
@@ -751,9 +754,9 @@ def oracle_sample_rate(w, sel, budget_s: float, rank_seed: int = 0, seg_offset: 
 
 def _pool_worker(job):
     """One host core of the all-cores oracle figure (run in a spawned process)."""
-    name, requests, layers, selector, budget_s, offset = job
+    name, requests, layers, beacons, selector, budget_s, offset = job
     import types
-    args = types.SimpleNamespace(workload=name, requests=requests, layers=layers, selector=selector)
+    args = types.SimpleNamespace(workload=name, requests=requests, layers=layers, beacons=beacons, selector=selector)
     w, sel = make_workload(args)
     t0 = time.perf_counter()
     rate, _, n_seg = oracle_sample_rate(w, sel, budget_s, rank_seed=offset, seg_offset=offset)
@@ -769,7 +772,8 @@ def oracle_pool_rate(args, budget_s: float):
     cores = len(os.sched_getaffinity(0))
     w, sel = make_workload(args)
     n_segs = w.num_requests * w.num_layers * w.num_kv_heads
-    jobs = [(args.workload, args.requests, args.layers, sel, budget_s, (i * n_segs) // cores)
+    jobs = [(args.workload, args.requests, args.layers, getattr(args, "beacons", None), sel, budget_s,
+             (i * n_segs) // cores)
             for i in range(cores)]
     # spawn (never fork after CUDA is initialised); a worker that dies raises
     # instead of leaving the pool waiting

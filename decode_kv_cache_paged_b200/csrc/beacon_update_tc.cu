@@ -434,18 +434,6 @@ __device__ __forceinline__ int64_t pipe_point(const BeaconUpdateParams &p, const
   return ((((int64_t)g.r * p.layers + g.l) * p.W + slot) * p.hq + (g.h * p.G + gq)) * 128;
 }
 
-// Distributed shared memory between the two CTAs of a cluster.
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// The same shared-memory offset in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
 // Asynchronous stores into the peer CTA's shared memory, each completing as
 // transaction bytes on a barrier of the peer (whose complete-tx releases the
 // bytes at cluster scope): no fence on the sending side.
@@ -484,9 +472,6 @@ __device__ __forceinline__ bool mbar_wait_cl(uint64_t *bar, uint32_t parity, vol
       return false;
     }
   }
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 
 // L2 prefetches: `bytes` contiguous bytes (16-byte aligned, a multiple of
@@ -728,12 +713,18 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           float v[32];
           tmem_ld32(tmem_base + lane_addr + ab * BM + c0, v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float dist = fmaf(-2.f, v[i], cnb[c0 + i]);
-            nan |= valid && (dist != dist);
-            if (dist < bst[i & 3]) {
-              bst[i & 3] = dist;
+          for (int i = 0; i < 32; i += 2) {
+            // two distances per packed FMA (each rounded as one fmaf)
+            const float2 cc = *reinterpret_cast<const float2 *>(cnb + c0 + i);
+            const float2 d2 = __ffma2_rn(make_float2(-2.f, -2.f), make_float2(v[i], v[i + 1]), cc);
+            nan |= valid && (d2.x != d2.x || d2.y != d2.y);
+            if (d2.x < bst[i & 3]) {
+              bst[i & 3] = d2.x;
               bix[i & 3] = c0 + i;
+            }
+            if (d2.y < bst[(i + 1) & 3]) {
+              bst[(i + 1) & 3] = d2.y;
+              bix[(i + 1) & 3] = c0 + i + 1;
             }
           }
         }
