@@ -434,6 +434,23 @@ __device__ __forceinline__ int64_t pipe_point(const BeaconUpdateParams &p, const
   return ((((int64_t)g.r * p.layers + g.l) * p.W + slot) * p.hq + (g.h * p.G + gq)) * 128;
 }
 
+// Distributed shared memory between the two CTAs of a cluster.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+// Every thread of both CTAs of the cluster arrives; neither goes on before
+// all have.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
 // Asynchronous stores into the peer CTA's shared memory, each completing as
 // transaction bytes on a barrier of the peer (whose complete-tx releases the
 // bytes at cluster scope): no fence on the sending side.
