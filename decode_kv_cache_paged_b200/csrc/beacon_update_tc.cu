@@ -519,7 +519,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   uint8_t *smem = smem_align<1024>(smem_raw);
   constexpr int D = 128;
   constexpr uint32_t kXBytes = 32768;    // 128 points x 128 bf16
-  constexpr uint32_t kCBytes = BM * 256;  // one term of one beacon buffer: [2 K-blocks][B rows][128 B]
+  constexpr uint32_t kCBytes = BM * 256;  // one term of one beacon buffer (B rows x 128 bf16)
+  // a beacon buffer holds, per 64-dimension block, the B hi rows followed by
+  // the B lo rows: [2 K-blocks][hi B rows | lo B rows][128 B], 128-byte
+  // swizzle; one assignment product per term
+  constexpr uint32_t kAsgCols = BM;          // TMEM columns of one assignment buffer
+  constexpr uint32_t kSumCol0 = 2 * kAsgCols;  // first sums column
+  constexpr uint32_t kTmemAlloc = 4u * BM;
   constexpr uint32_t kOHBytes = BM * 256; // one one-hot tile: [2 point blocks][B rows][128 B]
   // this CTA's beacons: [b_lo, b_lo + B) of the segment's Bg
   const int Bg = p.B;
@@ -528,9 +534,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   const int B = CL > 1 ? (rank ? Bg - 128 : 128) : Bg;
   const int seg0 = blockIdx.x / CL, seg_step = gridDim.x / CL;
   uint8_t *xs = smem;
-  uint8_t *chi = xs + NXS * kXBytes;
-  uint8_t *clo = chi + NCB * kCBytes;
-  uint8_t *oh = clo + NCB * kCBytes;
+  uint8_t *cterm = xs + NXS * kXBytes;  // [NCB][2 K-blocks][2 B rows][128 B]
+  uint8_t *oh = cterm + NCB * 2 * kCBytes;
   // squared norms: a ring of NCB + 2, so that the preparation of segment
   // si + NCB (which starts once the MMA has read segment si's terms) never
   // overwrites the norms of a segment the point warps may still scan
@@ -599,7 +604,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   fence_proxy_async();
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
-                 "r"(4 * BM));
+                 "r"(kTmemAlloc));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tmem_fence_before();
@@ -623,13 +628,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         if (!ok) return;
         tmem_fence_after();
         const uint32_t xa = smem_u32(xs + (gi % NXS) * kXBytes);
-        const uint32_t ha = smem_u32(chi + cb * kCBytes), la = smem_u32(clo + cb * kCBytes);
+        const uint32_t ca = smem_u32(cterm + cb * 2 * kCBytes);
         for (int term = 0; term < 2; ++term)
           for (int kb = 0; kb < 2; ++kb)
             for (int ks = 0; ks < 4; ++ks) {
               const uint64_t a = sw128_desc(xa + kb * 16384 + ks * 32);
-              const uint64_t bd = sw128_desc((term ? la : ha) + kb * B * 128 + ks * 32);
-              umma(tmem_base + (gi & 1) * BM, a, bd, idesc_asg, (term | kb | ks) != 0);
+              const uint64_t bd = sw128_desc(ca + kb * 2 * B * 128 + term * B * 128 + ks * 32);
+              umma(tmem_base + (gi & 1) * kAsgCols, a, bd, idesc_asg, (term | kb | ks) != 0);
             }
         umma_commit(&acc_full[gi & 1]);
         if (t == T - 1) umma_commit(&prep_empty[cb]);  // the beacon terms have been read
@@ -647,7 +652,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           uint64_t a = sw128_desc(xa + ks * 2048);
           a = (a & ~(uint64_t)(0x3FFFull << 16)) | ((uint64_t)(16384 >> 4) << 16);
           const uint64_t bd = sw128_desc(oa + (ks >> 2) * B * 128 + (ks & 3) * 32);
-          umma(tmem_base + 2 * BM + sb * BM, a, bd, idesc_sum, (t > 0 || ks > 0) ? 1u : 0u);
+          umma(tmem_base + kSumCol0 + sb * BM, a, bd, idesc_sum, (t > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit(&x_empty[gi % NXS]);
         umma_commit(&oh_empty[gi % NOH]);
@@ -662,8 +667,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       // within a segment; at a segment boundary the last sums go first, so
       // that the running mean of a segment never waits for the next
       // segment's beacon preparation
+      // each segment's descriptor is loaded a segment ahead (its latency hidden)
+      PipeSeg g_next = seg0 < n_segs ? pipe_seg(p, seg0) : PipeSeg{};
       for (int s = seg0; s < n_segs && ok; s += seg_step, ++si) {
-        const PipeSeg g = pipe_seg(p, s);
+        const PipeSeg g = g_next;
+        if (s + seg_step < n_segs) g_next = pipe_seg(p, s + seg_step);
         for (int t = 0; t < g.T && ok; ++t, ++gi) {
           if (have_prev && t == 0) sums(pg, ps, pt, pT);
           assign(gi, si, t, g.T);
@@ -698,8 +706,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       peer_full = map_peer(smem_u32(xch_full), rank ^ 1u);
       peer_empty = map_peer(smem_u32(xch_empty), rank ^ 1u);
     }
+    // each segment's descriptor is loaded a segment ahead (its latency hidden)
+    PipeSeg g_next = seg0 < n_segs ? pipe_seg(p, seg0) : PipeSeg{};
     for (int s = seg0; s < n_segs && ok; s += seg_step, ++si) {
-      const PipeSeg g = pipe_seg(p, s);
+      const PipeSeg g = g_next;
+      if (s + seg_step < n_segs) g_next = pipe_seg(p, s + seg_step);
       const int cb = si % NCB, kb3 = si % 3;
       ok = lanes_wait(&prep_full[cb], (si / NCB) & 1, abort_flag, p.status) &&
            lanes_wait(&cnt_empty[kb3], ((si / 3) & 1) ^ 1, abort_flag, p.status);
@@ -726,11 +737,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           bst[j] = __int_as_float(0x7f800000);
           bix[j] = 0;
         }
-        for (int c0 = 0; c0 < B; c0 += 32) {
-          float v[32];
-          tmem_ld32(tmem_base + lane_addr + ab * BM + c0, v);
+        constexpr int kChunk = 32;
+        for (int c0 = 0; c0 < B; c0 += kChunk) {
+          float v[kChunk];
+          tmem_ld32(tmem_base + lane_addr + ab * kAsgCols + c0, v);
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
+          for (int i = 0; i < kChunk; i += 2) {
             // two distances per packed FMA (each rounded as one fmaf)
             const float2 cc = *reinterpret_cast<const float2 *>(cnb + c0 + i);
             const float2 d2 = __ffma2_rn(make_float2(-2.f, -2.f), make_float2(v[i], v[i + 1]), cc);
@@ -812,11 +824,14 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     const int b = (warp - 5) * 32 + lane;
     int si = 0;
     bool ok = true;
+    // each segment's descriptor is loaded a segment ahead (its latency hidden)
+    PipeSeg g_next = seg0 < n_segs ? pipe_seg(p, seg0) : PipeSeg{};
     for (int s = seg0; s < n_segs && ok; s += seg_step, ++si) {
-      const PipeSeg g = pipe_seg(p, s);
+      const PipeSeg g = g_next;
+      if (s + seg_step < n_segs) g_next = pipe_seg(p, s + seg_step);
       const int cb = si % NCB;
       const bool have = b < B;
-      uint8_t *hb = chi + cb * kCBytes, *lb = clo + cb * kCBytes;
+      uint8_t *hb = cterm + cb * 2 * kCBytes, *lb = hb + B * 128;  // lo rows follow the hi rows
       const float *frow = p.beacons + (g.seg * Bg + b_lo + b) * D;
       const __nv_bfloat16 *irow =
           ring + pipe_point(p, g, (int)(((int64_t)(b_lo + (have ? b : 0)) * g.n_pts) / Bg));
@@ -842,7 +857,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       load_q(0);  // in flight while the buffer is still in use
       // the pair form: this CTA's beacons of its next segment into L2
       if (CL > 1 && b == 0 && s + seg_step < n_segs) {
-        const PipeSeg gn = pipe_seg(p, s + seg_step);
+        const PipeSeg &gn = g_next;
         prefetch_l2(p.beacons + (gn.seg * Bg + b_lo) * D, (uint32_t)(B * D * sizeof(float)));
       }
       // the old count, for the running mean a segment or two later
@@ -875,7 +890,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             l[e] = *reinterpret_cast<const uint32_t *>(&ll);
           }
           const int kk = kq * 32 + ch * 8;  // the chunk's first dimension
-          const uint32_t off = (uint32_t)(kk >> 6) * (uint32_t)B * 128u + sw128_off(b, kk & 63);
+          const uint32_t off = (uint32_t)(kk >> 6) * 2u * (uint32_t)B * 128u + sw128_off(b, kk & 63);
           *reinterpret_cast<uint4 *>(hb + off) = make_uint4(h[0], h[1], h[2], h[3]);
           *reinterpret_cast<uint4 *>(lb + off) = make_uint4(l[0], l[1], l[2], l[3]);
         }
@@ -896,12 +911,15 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       uint32_t gl = 0;
       bool ok = true;
       const int S = 128 / p.G;
+      // each segment's descriptor is loaded a segment ahead (its latency hidden)
+      PipeSeg g_next = seg0 < n_segs ? pipe_seg(p, seg0) : PipeSeg{};
       for (int s = seg0; s < n_segs && ok; s += seg_step) {
-        const PipeSeg g = pipe_seg(p, s);
+        const PipeSeg g = g_next;
+        if (s + seg_step < n_segs) g_next = pipe_seg(p, s + seg_step);
         const int z0 = (g.r * p.layers + g.l) * p.W;  // ring row of slot 0 of this (request, layer)
         // the pair form: the next segment's point tiles into L2 (one CTA)
         if (CL > 1 && rank == 0 && s + seg_step < n_segs) {
-          const PipeSeg gn = pipe_seg(p, s + seg_step);
+          const PipeSeg &gn = g_next;
           const int zn = (gn.r * p.layers + gn.l) * p.W;
           for (int t = 0; t < gn.T; ++t)
             for (int kb = 0; kb < 2; ++kb) prefetch_box_3d(&qmap, kb * 64, gn.h * p.G, zn + t * S);
@@ -933,8 +951,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     int si = 0;
     uint32_t ph = 0;
     bool ok = true;
+    // each segment's descriptor is loaded a segment ahead (its latency hidden)
+    PipeSeg g_next = seg0 < n_segs ? pipe_seg(p, seg0) : PipeSeg{};
     for (int s = seg0; s < n_segs && ok; s += seg_step, ++si) {
-      const PipeSeg g = pipe_seg(p, s);
+      const PipeSeg g = g_next;
+      if (s + seg_step < n_segs) g_next = pipe_seg(p, s + seg_step);
       const int kb3 = si % 3, sb = si & 1;
       int32_t *cntb = cnt + kb3 * BM;
       float *gbeac = p.beacons + (g.seg * Bg + b_lo) * D;
@@ -978,7 +999,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       if (!ok) break;
       for (int b0 = 0; b0 < B; b0 += 32) {
         float sm[32], v[32];
-        tmem_ld32(tmem_base + lane_addr + 2 * BM + sb * BM + b0, sm);
+        tmem_ld32(tmem_base + lane_addr + kSumCol0 + sb * BM + b0, sm);
 #pragma unroll
         for (int u = 0; u < 32; ++u) v[u] = onext[u];
         if (b0 + 32 < B) load_old(b0 + 32);
@@ -1005,7 +1026,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   if constexpr (CL > 1) cluster_sync_all();
   if (warp == 0) {
     tmem_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(4 * BM));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemAlloc));
   }
 }
 
