@@ -85,3 +85,30 @@ def test_committed_traffic_entries_are_well_formed():
             assert len(e["source_hash"]) == 16
             n += 1
     assert n >= 4
+
+
+def test_workload_overrides():
+    """--requests/--layers/--beacons reach the workload; a random selector drops the beacon state."""
+    import types
+    args = types.SimpleNamespace(workload="long_trace", requests=2, layers=4, beacons=128, selector=None)
+    w, sel = bench.make_workload(args)
+    assert (w.num_requests, w.num_layers, w.num_beacons, sel) == (2, 4, 128, "beacon")
+    assert len(w.length) == 2 and int(w.length[0]) == 32768
+    args = types.SimpleNamespace(workload="beacon_serving", requests=None, layers=None, beacons=None,
+                                 selector="random")
+    w, sel = bench.make_workload(args)
+    assert sel == "random" and w.num_beacons == 0 and w.query_window == 0
+
+
+def test_pool_jobs_carry_the_beacon_override(monkeypatch):
+    """The all-cores oracle rebuilds the workload in each worker from the job tuple: the beacon override
+    must travel with it."""
+    import types
+    seen = []
+
+    def fake_rate(w, sel, budget_s, rank_seed=0, seg_offset=0):
+        seen.append(w.num_beacons)
+        return 1.0, "", 1
+    monkeypatch.setattr(bench, "oracle_sample_rate", fake_rate)
+    bench._pool_worker(("long_trace", 1, 1, 64, "beacon", 0.01, 0))
+    assert seen == [64]
