@@ -9,6 +9,7 @@
 // one GPU; every byte of K/V and every score is produced by the kernels in the
 // other .cu files.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -18,6 +19,18 @@
 #include <vector>
 
 #include "kvc_internal.h"
+
+namespace {
+// NVTX range for the duration of a scope: the library's calls and the phases
+// of a round show up by name in profilers (ncu --nvtx --nvtx-include ...).
+// Without an attached tool each push and pop returns at once.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
+}  // namespace
 
 using namespace kvc;
 
@@ -386,6 +399,7 @@ kvc_status kvc_set_option(kvc_ctx *ctx, kvc_option opt, int64_t value) {
 
 kvc_status kvc_append(kvc_ctx *ctx, const int32_t *req_ids, int32_t n_req, int32_t n_tokens,
                       const void *k_new, const void *v_new, const void *q_new, int32_t protect) {
+  NvtxRange nvtx_range("kvc_append");
   if (!ctx) return KVC_ERR_INVALID_ARG;
   const kvc_config &c = ctx->cfg;
   if (n_req < 0 || n_tokens < 0) return fail(ctx, KVC_ERR_INVALID_ARG, "negative n_req or n_tokens");
@@ -485,6 +499,7 @@ kvc_status kvc_append(kvc_ctx *ctx, const int32_t *req_ids, int32_t n_req, int32
 }
 
 kvc_status kvc_update_beacons(kvc_ctx *ctx, int32_t *assign_out, float *ms_out) {
+  NvtxRange nvtx_range("kvc_update_beacons");
   if (!ctx) return KVC_ERR_INVALID_ARG;
   const kvc_config &c = ctx->cfg;
   if (c.num_beacons == 0) return fail(ctx, KVC_ERR_STATE, "the context has no beacon state (num_beacons = 0)");
@@ -555,6 +570,7 @@ kvc_status kvc_compress(kvc_ctx *ctx, kvc_selector selector, const int32_t *budg
 kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *budgets,
                            uint64_t seed, const kvc_round_options *opts, void *debug_scores,
                            kvc_round_stats *stats) {
+  NvtxRange nvtx_range("kvc_compress");
   if (!ctx) return KVC_ERR_INVALID_ARG;
   const kvc_config &c = ctx->cfg;
   if (selector != KVC_SEL_RANDOM && selector != KVC_SEL_RANDOM_SHARED && selector != KVC_SEL_BEACON &&
@@ -627,6 +643,7 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
   cudaError_t e;
   float *score_buf = (debug_scores && beacon_sel) ? static_cast<float *>(debug_scores) : ctx->d_scores;
   if (beacon_sel && !segs.empty()) {
+    NvtxRange nvtx_score("score");  // inside kvc_compress: "kvc_compress/score/" to ncu
     BeaconScoreParams bp{};
     bp.k_pool = ctx->k_pool;
     bp.block_table = ctx->d_bt;
@@ -678,22 +695,25 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
   const int mode = selector == KVC_SEL_RANDOM ? kModeRandom
                    : selector == KVC_SEL_RANDOM_SHARED ? kModeRandomShared : kModeScores;
   // buckets: candidate counts up to 2^k
-  size_t i0 = 0;
-  while (i0 < segs.size()) {
-    int cap = 1024;
-    while (cap < segs[i0].L - segs[i0].P) cap *= 2;
-    size_t i1 = i0;
-    int max_m = 0;
-    while (i1 < segs.size() && segs[i1].L - segs[i1].P <= cap) {
-      max_m = std::max(max_m, segs[i1].M);
-      ++i1;
+  {
+    NvtxRange nvtx_select("select_compact");  // "kvc_compress/select_compact/"
+    size_t i0 = 0;
+    while (i0 < segs.size()) {
+      int cap = 1024;
+      while (cap < segs[i0].L - segs[i0].P) cap *= 2;
+      size_t i1 = i0;
+      int max_m = 0;
+      while (i1 < segs.size() && segs[i1].L - segs[i1].P <= cap) {
+        max_m = std::max(max_m, segs[i1].M);
+        ++i1;
+      }
+      const int max_n = segs[i1 - 1].L - segs[i1 - 1].P;
+      sp.segs = d_segs + i0;
+      e = launch_select_compact(sp, mode, (int)(i1 - i0), max_n, max_m, ctx->stream);
+      if (e != cudaSuccess) return cuda_fail(ctx, e, "select_compact");
+      st.launches += 1;
+      i0 = i1;
     }
-    const int max_n = segs[i1 - 1].L - segs[i1 - 1].P;
-    sp.segs = d_segs + i0;
-    e = launch_select_compact(sp, mode, (int)(i1 - i0), max_n, max_m, ctx->stream);
-    if (e != cudaSuccess) return cuda_fail(ctx, e, "select_compact");
-    st.launches += 1;
-    i0 = i1;
   }
   if (timed) KVC_CUDA(ctx, cudaEventRecord(ctx->ev[2], ctx->stream));
   KVC_CUDA(ctx, cudaMemcpyAsync(ctx->d_len, sd_stage.d + align_up(seg_bytes, 16), (size_t)R * 4,
@@ -763,6 +783,7 @@ kvc_status kvc_get_lengths(const kvc_ctx *ctx, int32_t *lengths, int32_t *prompt
 
 kvc_status kvc_gather_dense(kvc_ctx *ctx, int32_t layer, int32_t req_begin, int32_t req_count,
                             int32_t cap, void *k_out, void *v_out, int32_t *pos_out) {
+  NvtxRange nvtx_range("kvc_gather_dense");
   if (!ctx) return KVC_ERR_INVALID_ARG;
   const kvc_config &c = ctx->cfg;
   if (layer < 0 || layer >= c.num_layers || req_begin < 0 || req_count < 0 ||
@@ -784,6 +805,7 @@ kvc_status kvc_gather_dense(kvc_ctx *ctx, int32_t layer, int32_t req_begin, int3
 
 kvc_status kvc_decode_attention(kvc_ctx *ctx, int32_t layer_begin, int32_t layer_count, const void *q,
                                 float scale, float *out, float *lse, float *ms_out) {
+  NvtxRange nvtx_range("kvc_decode_attention");
   if (!ctx) return KVC_ERR_INVALID_ARG;
   const kvc_config &c = ctx->cfg;
   if (layer_begin < 0 || layer_count < 1 || layer_begin + layer_count > c.num_layers)
