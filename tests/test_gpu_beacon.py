@@ -336,9 +336,11 @@ def test_tcgen05_logit_far_above_running_max(B):
 
 @pytest.mark.parametrize("impl,B,W,Hq", [(1, 64, 64, 32), (2, 64, 64, 32), (2, 32, 64, 32), (2, 96, 64, 32),
                                          (2, 128, 64, 32), (2, 256, 64, 32), (2, 64, 40, 32), (2, 64, 50, 16),
-                                         (2, 192, 64, 32), (2, 160, 100, 16), (2, 256, 256, 32)],
+                                         (2, 192, 64, 32), (2, 160, 100, 16), (2, 256, 256, 32),
+                                         (2, 64, 64, 24), (2, 256, 96, 24)],
                          ids=["simt-64", "tc-64", "tc-32", "tc-96", "tc-128", "tc-256", "tc-64-160pts",
-                              "tc-64-G2-100pts", "tc-192", "tc-160-G2-200pts", "tc-256-1024pts"])
+                              "tc-64-G2-100pts", "tc-192", "tc-160-G2-200pts", "tc-256-1024pts",
+                              "tc-64-G3", "tc-256-G3"])
 def test_second_update_against_oracle(impl, B, W, Hq):
     """A later (non-initial) update: fp32 beacons with counts, new points.
     The oracle recomputes it from the GPU's beacons and counts before the
@@ -348,7 +350,8 @@ def test_second_update_against_oracle(impl, B, W, Hq):
     leave the last 128-point tile partly filled (160 points; G = 2 with 100
     points, a single partial tile).  More than 128 beacons split over a CTA
     pair: 192 and 160 (second halves of 64 and 32 beacons, the latter with a
-    partial last tile) and 256 over the long trace's 1024-point window."""
+    partial last tile) and 256 over the long trace's 1024-point window.  G = 3 (24 query heads) does not
+    divide a 128-point tile into whole ring slots: those updates take the one-CTA-per-segment kernel."""
     w = wl.beacon_serving(R=2, layers=2)
     w.num_beacons = B
     w.num_q_heads = Hq
