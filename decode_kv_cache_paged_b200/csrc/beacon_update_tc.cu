@@ -347,8 +347,8 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
 
 
 // ---------------------------------------------------------------------------
-// Pipelined form for up to 128 beacons.  One persistent CTA per SM walks its
-// segments; the work is split by role so that the point loads, the beacon
+// Pipelined form (a CTA pair per segment above 128 beacons, below).  One
+// persistent CTA per SM walks its segments; the work is split by role so that the point loads, the beacon
 // preparation, the products, the argmins and the running means of
 // neighbouring tiles and segments overlap instead of running as one serial
 // chain per segment:
@@ -357,8 +357,9 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
 //               the sums of tile g, and a segment's last sums before the next
 //               segment's first assignment;
 //   warps 1-4   point warps: one point per thread: the argmin over its TMEM
-//               lane of the assignment product, its one-hot entry and its
-//               count;
+//               lane of the assignment product (four interleaved compare
+//               chains, merged by value then index), its one-hot entry and
+//               its count;
 //   warps 5-8   preparation, one beacon per thread: the next segment's
 //               beacons as bf16 hi/lo terms (swizzled, the B operand of the
 //               assignment) and their fp32 squared norms;
@@ -385,7 +386,9 @@ __global__ void __launch_bounds__(kUT) beacon_update_tc_kernel(BeaconUpdateParam
 // (sums of neighbouring segments alternate).  NOH one-hot tiles: two, or one
 // where shared memory is better spent on a third point stage.  The counts of
 // three segments rotate in shared memory so that the preparation never waits
-// for a mean.
+// for a mean, and the squared norms through NCB + 2 buffers so that it waits
+// only for the MMA's last read of the beacon terms.  Every role loads the
+// next segment's descriptor a segment ahead.
 // More than 128 beacons: a cluster of two CTAs per segment (CL = 2), CTA r
 // holding beacons [128 r, 128 r + nb) with the layout above.  Both load the
 // same point tiles; each point thread takes the argmin over its CTA's
