@@ -623,9 +623,10 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
   }
   if (beacon_sel && c.num_beacons == 0)
     return fail(ctx, KVC_ERR_STATE, "the context has no beacon state (num_beacons = 0)");
-  // bucket by candidate count so each launch sizes its shared memory to its segments
+  // longest first (the persistent select launch takes its segments in list
+  // order), bucketed by candidate count so each launch sizes its shared memory
   std::stable_sort(segs.begin(), segs.end(), [](const SegDesc &a, const SegDesc &b) {
-    return (a.L - a.P) < (b.L - b.P);
+    return (a.L - a.P) > (b.L - b.P);
   });
   const size_t seg_bytes = segs.size() * sizeof(SegDesc);
   Stage sd_stage;
@@ -694,20 +695,28 @@ kvc_status kvc_compress_ex(kvc_ctx *ctx, kvc_selector selector, const int32_t *b
   sp.round = (uint64_t)ctx->round;
   const int mode = selector == KVC_SEL_RANDOM ? kModeRandom
                    : selector == KVC_SEL_RANDOM_SHARED ? kModeRandomShared : kModeScores;
-  // buckets: candidate counts up to 2^k
+  // launches: every segment with more than kSelectSmallMax candidates in one
+  // (the kernel's persistent form, which balances the segments itself), the
+  // others in buckets of candidate counts (2^(k-1), 2^k], k >= 10.  The split
+  // only sizes the launches: any bucket is computed correctly.
   {
     NvtxRange nvtx_select("select_compact");  // "kvc_compress/select_compact/"
+    constexpr int kSelectSmallMax = 4096;
     size_t i0 = 0;
     while (i0 < segs.size()) {
-      int cap = 1024;
-      while (cap < segs[i0].L - segs[i0].P) cap *= 2;
+      const int max_n = segs[i0].L - segs[i0].P;
+      int lo = kSelectSmallMax;
+      if (max_n <= kSelectSmallMax) {
+        int cap = 1024;
+        while (cap < max_n) cap *= 2;
+        lo = cap == 1024 ? 0 : cap / 2;
+      }
       size_t i1 = i0;
       int max_m = 0;
-      while (i1 < segs.size() && segs[i1].L - segs[i1].P <= cap) {
+      while (i1 < segs.size() && segs[i1].L - segs[i1].P > lo) {
         max_m = std::max(max_m, segs[i1].M);
         ++i1;
       }
-      const int max_n = segs[i1 - 1].L - segs[i1 - 1].P;
       sp.segs = d_segs + i0;
       e = launch_select_compact(sp, mode, (int)(i1 - i0), max_n, max_m, ctx->stream);
       if (e != cudaSuccess) return cuda_fail(ctx, e, "select_compact");

@@ -214,74 +214,187 @@ __device__ __forceinline__ int block_scan_each(int lo, int hi, Pred pred, Fn fn,
   return tot;
 }
 
+// One (request, layer, KV head) segment of a launch: item i of the launch is
+// request segs[i / (hkv * layers)], layer (i / hkv) % layers, head i % hkv.
+struct ScSeg {
+  int h, l, r, P, M, N;
+  const int32_t *bt;
+  int64_t layer_page0, seg_flat;
+};
+
+__device__ __forceinline__ ScSeg sc_seg(const SelectCompactParams &p, int item) {
+  ScSeg g;
+  g.h = item % p.hkv;
+  g.l = (item / p.hkv) % p.layers;
+  const SegDesc sd = p.segs[item / (p.hkv * p.layers)];
+  g.r = sd.req;
+  g.P = sd.P;
+  g.M = sd.M;
+  g.N = sd.L - sd.P;
+  g.bt = p.block_table + (int64_t)g.r * p.bt_stride;
+  g.layer_page0 = (int64_t)g.l * p.num_pages;
+  g.seg_flat = ((int64_t)g.r * p.layers + g.l) * p.hkv + g.h;
+  return g;
+}
+
+// global row index (also the position-map index) of slot s of the segment
+__device__ __forceinline__ int64_t sc_row(const SelectCompactParams &p, const ScSeg &g, int s) {
+  return ((g.layer_page0 + g.bt[s >> 4]) * p.hkv + g.h) * kPage + (s & (kPage - 1));
+}
+
+// 32-bit ranking key of candidate j (slot P + j): the order key of the beacon
+// score, or the high word of the Philox draw of (position / block, head,
+// layer, request) under (seed, round)
+template <int MODE>
+__device__ __forceinline__ uint32_t sc_key(const SelectCompactParams &p, const ScSeg &g, int j) {
+  if (MODE == kModeScores) return float_order_key(p.scores[g.seg_flat * p.max_seq + j]);
+  const uint64_t head_field = (MODE == kModeRandomShared) ? ~0ull : (uint64_t)g.h;
+  const int pos = p.pos_map[sc_row(p, g, g.P + j)];
+  const uint32_t key = philox4x64_10_word0_hi32((uint64_t)(int64_t)(pos / p.block), head_field, (uint64_t)g.l,
+                                                (uint64_t)g.r, p.seed, p.round);
+  if (p.debug) p.debug[g.seg_flat * p.max_seq + j] = key;
+  return key;
+}
+
+// Shared scratch of the select and rank steps.
+template <int NT>
+struct ScScratch {
+  uint32_t hist[256];
+  uint32_t bcast[4];
+  uint32_t cand[kFinish];
+  uint32_t warp_cnt[NT / 32], warp_eq[NT / 32];
+  int first_evicted;
+  int next;  // persistent form: the next work item
+};
+
+// The survivors' threshold: keys above tau stay; of the count_eq keys equal
+// to tau, `need` stay -- the lowest slots, or (split_by_pos) the lowest
+// positions, those whose complemented position is at least ptau.
+struct ScThreshold {
+  uint32_t tau, ptau;
+  int need, count_eq;
+  bool split_by_pos;
+};
+
+template <int NT, int VAR>
+__device__ __forceinline__ ScThreshold sc_threshold(const SelectCompactParams &p, const ScSeg &g,
+                                                    const uint32_t *keys, ScScratch<NT> &sh) {
+  ScThreshold t;
+  block_radix_select<NT>(
+      g.N, g.M, [&](int j, uint32_t &k) { k = keys[j]; return true; }, sh.hist, sh.bcast, sh.cand, t.tau, t.need,
+      t.count_eq);
+  // with ties split and slots possibly out of position order: the `need`
+  // lowest positions among the tied keys (positions are distinct)
+  t.ptau = 0;
+  t.split_by_pos = VAR != kOrderedSlotTie && t.need < t.count_eq;
+  if (t.split_by_pos) {
+    int need2, cnt2;
+    const uint32_t tau = t.tau;
+    block_radix_select<NT>(
+        g.N, t.need,
+        [&](int j, uint32_t &k) {
+          if (keys[j] != tau) return false;
+          k = ~(uint32_t)p.pos_map[sc_row(p, g, g.P + j)];
+          return true;
+        },
+        sh.hist, sh.bcast, sh.cand, t.ptau, need2, cnt2);
+  }
+  return t;
+}
+
+// kept flag of candidate j when ties go by position
+__device__ __forceinline__ bool sc_kept_pos(const SelectCompactParams &p, const ScSeg &g, const uint32_t *keys,
+                                            const ScThreshold &t, int j) {
+  const uint32_t key = keys[j];
+  if (key != t.tau) return key > t.tau;
+  if (!t.split_by_pos) return true;
+  return ~(uint32_t)p.pos_map[sc_row(p, g, g.P + j)] >= t.ptau;
+}
+
+// Ranks of an order-preserving round: src_of_rank[q] = the candidate that
+// becomes the q-th survivor, for q < M, and the first evicted candidate in
+// sh.first_evicted (N if none).  Ends with a block barrier.
+template <int NT, int VAR>
+__device__ __forceinline__ void sc_ordered_ranks(const SelectCompactParams &p, const ScSeg &g, const uint32_t *keys,
+                                                 const ScThreshold &t, uint16_t *src_of_rank, ScScratch<NT> &sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int N = g.N;
+  if (VAR == kOrderedSlotTie) {
+    // kept = key > tau, or key == tau among the first `need` such slots:
+    // two counts per candidate (greater, equal) scanned over warp ranges
+    constexpr int NW = NT / 32;
+    const uint32_t tau = t.tau;
+    const int need = t.need;
+    const int per = ((N + NW * 32 - 1) / (NW * 32)) * 32;
+    const int w0 = warp * per, w1 = min(N, w0 + per);
+    int cgt = 0, ceq = 0;
+    for (int base = w0; base < w1; base += 32) {
+      const int j = base + lane;
+      const uint32_t key = j < w1 ? keys[j] : 0u;
+      cgt += __popc(__ballot_sync(0xffffffffu, j < w1 && key > tau));
+      ceq += __popc(__ballot_sync(0xffffffffu, j < w1 && key == tau));
+    }
+    if (lane == 0) {
+      sh.warp_cnt[warp] = cgt;
+      sh.warp_eq[warp] = ceq;
+    }
+    __syncthreads();
+    int off_gt = 0, off_eq = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      if (w < warp) {
+        off_gt += sh.warp_cnt[w];
+        off_eq += sh.warp_eq[w];
+      }
+    }
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int base = w0; base < w1; base += 32) {
+      const int j = base + lane;
+      const bool valid = j < w1;
+      const uint32_t key = valid ? keys[j] : 0u;
+      const bool gt = valid && key > tau;
+      const bool eq = valid && key == tau;
+      const unsigned mgt = __ballot_sync(0xffffffffu, gt);
+      const unsigned meq = __ballot_sync(0xffffffffu, eq);
+      const int gt_before = off_gt + __popc(mgt & lt_mask);
+      const int eq_before = off_eq + __popc(meq & lt_mask);
+      const bool kept = gt || (eq && eq_before < need);
+      if (kept) {
+        src_of_rank[gt_before + min(eq_before, need)] = (uint16_t)j;
+      } else if (valid) {
+        atomicMin(&sh.first_evicted, j);
+      }
+      off_gt += __popc(mgt);
+      off_eq += __popc(meq);
+    }
+  } else {
+    block_scan_each<NT>(
+        0, N, [&](int j) { return sc_kept_pos(p, g, keys, t, j); },
+        [&](int j, int rank) { src_of_rank[rank] = (uint16_t)j; }, sh.warp_cnt);
+    for (int j = threadIdx.x; j < N; j += NT)
+      if (!sc_kept_pos(p, g, keys, t, j)) atomicMin(&sh.first_evicted, j);
+  }
+  __syncthreads();
+}
+
 template <int NT, int MODE, int kUnroll, int VAR>
 __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams p, int keys_cap) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint32_t *keys = reinterpret_cast<uint32_t *>(smem);                  // [keys_cap]
   uint16_t *src_of_rank = reinterpret_cast<uint16_t *>(keys + keys_cap);  // [keys_cap]
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t bcast[4];
-  __shared__ uint32_t cand[kFinish];
-  __shared__ uint32_t warp_cnt[NT / 32], warp_eq[NT / 32];
-  __shared__ int first_evicted;
+  __shared__ ScScratch<NT> sh;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int h = blockIdx.x % p.hkv;
-  const int l = (blockIdx.x / p.hkv) % p.layers;
-  const SegDesc sd = p.segs[blockIdx.x / (p.hkv * p.layers)];
-  const int r = sd.req, P = sd.P, M = sd.M;
-  const int N = sd.L - P;
-  const int32_t *bt = p.block_table + (int64_t)r * p.bt_stride;
-  const int64_t layer_page0 = (int64_t)l * p.num_pages;
-  const int64_t seg_flat = ((int64_t)r * p.layers + l) * p.hkv + h;
-  // global row index (also the position-map index) of slot s of this segment
-  auto row_of = [&](int s) -> int64_t {
-    return ((layer_page0 + bt[s >> 4]) * p.hkv + h) * kPage + (s & (kPage - 1));
-  };
+  const int tid = threadIdx.x;
+  const ScSeg g = sc_seg(p, blockIdx.x);
+  const int P = g.P, M = g.M, N = g.N;
 
   // 1. keys
-  if (tid == 0) first_evicted = N;
-  const uint64_t head_field = (MODE == kModeRandomShared) ? ~0ull : (uint64_t)h;
-  for (int j = tid; j < N; j += NT) {
-    uint32_t key;
-    if (MODE == kModeScores) {
-      key = float_order_key(p.scores[seg_flat * p.max_seq + j]);
-    } else {
-      const int pos = p.pos_map[row_of(P + j)];
-      key = philox4x64_10_word0_hi32((uint64_t)(int64_t)(pos / p.block), head_field, (uint64_t)l,
-                                     (uint64_t)r, p.seed, p.round);
-      if (p.debug) p.debug[seg_flat * p.max_seq + j] = key;
-    }
-    keys[j] = key;
-  }
+  if (tid == 0) sh.first_evicted = N;
+  for (int j = tid; j < N; j += NT) keys[j] = sc_key<MODE>(p, g, j);
   __syncthreads();
 
   // 2. threshold
-  uint32_t tau;
-  int need, count_eq;
-  block_radix_select<NT>(
-      N, M, [&](int j, uint32_t &k) { k = keys[j]; return true; }, hist, bcast, cand, tau, need, count_eq);
-  // with ties split and slots possibly out of position order: the `need`
-  // lowest positions among the tied keys (positions are distinct)
-  uint32_t ptau = 0;
-  const bool split_by_pos = VAR != kOrderedSlotTie && need < count_eq;
-  if (split_by_pos) {
-    int need2, cnt2;
-    block_radix_select<NT>(
-        N, need,
-        [&](int j, uint32_t &k) {
-          if (keys[j] != tau) return false;
-          k = ~(uint32_t)p.pos_map[row_of(P + j)];
-          return true;
-        },
-        hist, bcast, cand, ptau, need2, cnt2);
-  }
-  auto kept_pos = [&](int j) -> bool {  // kept flag when ties go by position
-    const uint32_t key = keys[j];
-    if (key != tau) return key > tau;
-    if (!split_by_pos) return true;
-    return ~(uint32_t)p.pos_map[row_of(P + j)] >= ptau;
-  };
+  const ScThreshold t = sc_threshold<NT, VAR>(p, g, keys, sh);
 
   const int vpr = p.row_bytes >> 4;  // 16-byte vectors per row
   const int rows_per_pass = NT / vpr;
@@ -291,63 +404,10 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
 
   if (VAR != kHoleFill) {
     // 3. ranks in slot order
-    if (VAR == kOrderedSlotTie) {
-      // kept = key > tau, or key == tau among the first `need` such slots:
-      // two counts per candidate (greater, equal) scanned over warp ranges
-      constexpr int NW = NT / 32;
-      const int per = ((N + NW * 32 - 1) / (NW * 32)) * 32;
-      const int w0 = warp * per, w1 = min(N, w0 + per);
-      int cgt = 0, ceq = 0;
-      for (int base = w0; base < w1; base += 32) {
-        const int j = base + lane;
-        const uint32_t key = j < w1 ? keys[j] : 0u;
-        cgt += __popc(__ballot_sync(0xffffffffu, j < w1 && key > tau));
-        ceq += __popc(__ballot_sync(0xffffffffu, j < w1 && key == tau));
-      }
-      if (lane == 0) {
-        warp_cnt[warp] = cgt;
-        warp_eq[warp] = ceq;
-      }
-      __syncthreads();
-      int off_gt = 0, off_eq = 0;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        if (w < warp) {
-          off_gt += warp_cnt[w];
-          off_eq += warp_eq[w];
-        }
-      }
-      const unsigned lt_mask = (1u << lane) - 1u;
-      for (int base = w0; base < w1; base += 32) {
-        const int j = base + lane;
-        const bool valid = j < w1;
-        const uint32_t key = valid ? keys[j] : 0u;
-        const bool gt = valid && key > tau;
-        const bool eq = valid && key == tau;
-        const unsigned mgt = __ballot_sync(0xffffffffu, gt);
-        const unsigned meq = __ballot_sync(0xffffffffu, eq);
-        const int gt_before = off_gt + __popc(mgt & lt_mask);
-        const int eq_before = off_eq + __popc(meq & lt_mask);
-        const bool kept = gt || (eq && eq_before < need);
-        if (kept) {
-          src_of_rank[gt_before + min(eq_before, need)] = (uint16_t)j;
-        } else if (valid) {
-          atomicMin(&first_evicted, j);
-        }
-        off_gt += __popc(mgt);
-        off_eq += __popc(meq);
-      }
-    } else {
-      block_scan_each<NT>(
-          0, N, [&](int j) { return kept_pos(j); },
-          [&](int j, int rank) { src_of_rank[rank] = (uint16_t)j; }, warp_cnt);
-      for (int j = tid; j < N; j += NT)
-        if (!kept_pos(j)) atomicMin(&first_evicted, j);
-    }
-    __syncthreads();
+    sc_ordered_ranks<NT, VAR>(p, g, keys, t, src_of_rank, sh);
 
     // 4. in-place, order-preserving copy of ranks [first_evicted, M)
-    const int q0 = first_evicted;
+    const int q0 = sh.first_evicted;
 #pragma unroll 1
     for (int base = q0; base < M; base += rows_per_pass * kUnroll) {
       uint4 kr[kUnroll], vr[kUnroll];
@@ -358,8 +418,8 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
         const int q = base + u * rows_per_pass + my_row;
         drow[u] = -1;
         if (active && q < M) {
-          const int64_t srow = row_of(P + src_of_rank[q]);
-          drow[u] = row_of(P + q);
+          const int64_t srow = sc_row(p, g, P + src_of_rank[q]);
+          drow[u] = sc_row(p, g, P + q);
           kr[u] = *reinterpret_cast<const uint4 *>(p.k_pool + srow * rb + my_vec * 16);
           vr[u] = *reinterpret_cast<const uint4 *>(p.v_pool + srow * rb + my_vec * 16);
           if (my_vec == 0) pr[u] = p.pos_map[srow];
@@ -381,11 +441,11 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
     // each listed in candidate order: holes at src_of_rank[0..), movers at
     // src_of_rank[M..)
     const int n_holes = block_scan_each<NT>(
-        0, M, [&](int j) { return !kept_pos(j); },
-        [&](int j, int i) { src_of_rank[i] = (uint16_t)j; }, warp_cnt);
+        0, M, [&](int j) { return !sc_kept_pos(p, g, keys, t, j); },
+        [&](int j, int i) { src_of_rank[i] = (uint16_t)j; }, sh.warp_cnt);
     block_scan_each<NT>(
-        M, N, [&](int j) { return kept_pos(j); },
-        [&](int j, int i) { src_of_rank[M + i] = (uint16_t)j; }, warp_cnt);
+        M, N, [&](int j) { return sc_kept_pos(p, g, keys, t, j); },
+        [&](int j, int i) { src_of_rank[M + i] = (uint16_t)j; }, sh.warp_cnt);
     __syncthreads();
     // 4'. the i-th mover goes to the i-th hole; all copies are independent
 #pragma unroll 1
@@ -398,8 +458,8 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
         const int i = base + u * rows_per_pass + my_row;
         drow[u] = -1;
         if (active && i < n_holes) {
-          const int64_t srow = row_of(P + src_of_rank[M + i]);
-          drow[u] = row_of(P + src_of_rank[i]);
+          const int64_t srow = sc_row(p, g, P + src_of_rank[M + i]);
+          drow[u] = sc_row(p, g, P + src_of_rank[i]);
           kr[u] = *reinterpret_cast<const uint4 *>(p.k_pool + srow * rb + my_vec * 16);
           vr[u] = *reinterpret_cast<const uint4 *>(p.v_pool + srow * rb + my_vec * 16);
           if (my_vec == 0) pr[u] = p.pos_map[srow];
@@ -418,6 +478,182 @@ __global__ void __launch_bounds__(NT) select_compact_kernel(SelectCompactParams 
   }
 }
 
+// Asynchronous 4-byte global -> shared copies (no register destination):
+// each thread waits only for the copies it issued itself.
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// The key of candidate j from the raw word fetched for it: the score's bits
+// (kModeScores) or its position (random selectors).
+template <int MODE>
+__device__ __forceinline__ uint32_t sc_key_from(const SelectCompactParams &p, const ScSeg &g, int j, uint32_t raw) {
+  if (MODE == kModeScores) return float_order_key(__uint_as_float(raw));
+  const uint64_t head_field = (MODE == kModeRandomShared) ? ~0ull : (uint64_t)g.h;
+  const uint32_t key = philox4x64_10_word0_hi32((uint64_t)(int64_t)((int)raw / p.block), head_field, (uint64_t)g.l,
+                                                (uint64_t)g.r, p.seed, p.round);
+  if (p.debug) p.debug[g.seg_flat * p.max_seq + j] = key;
+  return key;
+}
+
+// The persistent form's work counter: an int in the context's 256-byte
+// counter block, past the moved-row counter (zeroed before each launch).
+__host__ __device__ __forceinline__ int *sc_work_counter(const SelectCompactParams &p) {
+  return reinterpret_cast<int *>(p.counters + 24);
+}
+
+// Persistent form of the order-preserving round for segments with more than
+// 4096 candidates (one 512-thread CTA per SM, shared memory for up to 32768
+// candidates and two block-table rows).  Each CTA takes its segments from a
+// work counter, the list being ordered by decreasing candidate count
+// (longest first), and prepares the keys of its next segment during the copy
+// of the current one, so that the key draws (bound by the integer
+// multiplier) overlap the copy (bound by HBM) and only the threshold and the
+// ranks stay between two segments' copies:
+//   - before chunk 0, cp.async brings the next segment's block-table row
+//     (and, for beacon scores, the scores themselves) into shared memory;
+//   - after chunk 0's barrier has made that row visible, cp.async brings the
+//     position of every candidate (random selectors) into the keys buffer;
+//   - from the next chunk on, between issuing the chunk's loads and its
+//     barrier, each thread turns a share of the words it fetched itself into
+//     keys (Philox draws, or the scores' order keys).
+// No dependent global load sits between a chunk's loads and its stores, so
+// the draws never wait behind the copy's loads in flight.  The keys buffer is
+// free during the copy (the copy reads only src_of_rank), and the next
+// segment's rows are disjoint from the current one's.  The block-table rows
+// in shared memory also serve every row address of the copy.
+template <int MODE, int kUnroll, int VAR>
+__global__ void __launch_bounds__(512, 1)
+    select_compact_pipe_kernel(SelectCompactParams p, int n_items, int keys_cap, int m_cap) {
+  constexpr int NT = 512;
+  // draws start at this chunk: scores arrive with the block-table row, the
+  // positions of the random selectors one chunk later
+  constexpr int kFirst = MODE == kModeScores ? 1 : 2;
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint32_t *keys = reinterpret_cast<uint32_t *>(smem);                      // [keys_cap]
+  uint16_t *src_of_rank = reinterpret_cast<uint16_t *>(keys + keys_cap);      // [m_cap]
+  int32_t *bt_buf = reinterpret_cast<int32_t *>(src_of_rank + m_cap);         // [2][bt_stride]
+  __shared__ ScScratch<NT> sh;
+
+  const int tid = threadIdx.x;
+  int *work = sc_work_counter(p);
+  if (tid == 0) sh.next = atomicAdd(work, 1);
+  __syncthreads();
+  int cur = sh.next;
+  if (cur >= n_items) return;
+  ScSeg g = sc_seg(p, cur);
+  int buf = 0;
+  {
+    const int pages = (g.P + g.N + kPage - 1) / kPage;
+    for (int i = tid; i < pages; i += NT) bt_buf[i] = g.bt[i];
+    g.bt = bt_buf;
+    __syncthreads();
+    for (int j = tid; j < g.N; j += NT) keys[j] = sc_key<MODE>(p, g, j);
+  }
+
+  const int vpr = p.row_bytes >> 4;  // 16-byte vectors per row
+  const int rows_per_pass = NT / vpr;
+  const int rows_per_chunk = rows_per_pass * kUnroll;
+  const int my_row = tid / vpr, my_vec = tid - (tid / vpr) * vpr;
+  const bool active = my_row < rows_per_pass;
+  const int64_t rb = p.row_bytes;
+
+#pragma unroll 1
+  while (true) {
+    if (tid == 0) sh.first_evicted = g.N;
+    __syncthreads();  // the keys of g are complete
+    const ScThreshold t = sc_threshold<NT, VAR>(p, g, keys, sh);
+    sc_ordered_ranks<NT, VAR>(p, g, keys, t, src_of_rank, sh);
+    const int q0 = sh.first_evicted;
+    // the next item; every thread has read sh.next of the previous one and
+    // sh.first_evicted of this one before the barrier
+    if (tid == 0) sh.next = atomicAdd(work, 1);
+    __syncthreads();
+    const int nxt = sh.next;
+    const bool more = nxt < n_items;
+    ScSeg gn{};
+    int nn = 0;
+    int32_t *bt_next = bt_buf + (buf ^ 1) * p.bt_stride;
+    if (more) {
+      gn = sc_seg(p, nxt);
+      nn = gn.N;
+      const int pages = (gn.P + nn + kPage - 1) / kPage;
+      for (int i = tid; i < pages; i += NT) cp_async4(bt_next + i, gn.bt + i);
+      if (MODE == kModeScores) {
+        const float *src = p.scores + gn.seg_flat * p.max_seq;
+        for (int j = tid; j < nn; j += NT) cp_async4(keys + j, src + j);
+      }
+      cp_async_commit();
+      gn.bt = bt_next;  // read only once chunk 0's barrier (or the tail's) has made it visible
+    }
+    // positions of the next segment's candidates (random selectors)
+    auto fetch_positions = [&]() {
+      if (MODE != kModeScores) {
+        for (int j = tid; j < nn; j += NT) cp_async4(keys + j, p.pos_map + sc_row(p, gn, gn.P + j));
+        cp_async_commit();
+      }
+    };
+    const int M = g.M, P = g.P;
+    const int nchunks = M > q0 ? (M - q0 + rows_per_chunk - 1) / rows_per_chunk : 0;
+    const int per = nchunks > kFirst ? (nn + NT * (nchunks - kFirst) - 1) / (NT * (nchunks - kFirst)) : 0;
+    int jn = tid;  // this thread's next key of the next segment
+#pragma unroll 1
+    for (int c = 0, base = q0; base < M; ++c, base += rows_per_chunk) {
+      uint4 kr[kUnroll], vr[kUnroll];
+      int pr[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int q = base + u * rows_per_pass + my_row;
+        if (active && q < M) {
+          const int64_t srow = sc_row(p, g, P + src_of_rank[q]);
+          kr[u] = *reinterpret_cast<const uint4 *>(p.k_pool + srow * rb + my_vec * 16);
+          vr[u] = *reinterpret_cast<const uint4 *>(p.v_pool + srow * rb + my_vec * 16);
+          if (my_vec == 0) pr[u] = p.pos_map[srow];
+        }
+      }
+      if (c == 0) {
+        cp_async_wait_all();  // this thread's share of the row (and scores)
+      } else if (c == 1) {
+        fetch_positions();
+      }
+      if (c >= kFirst) {
+        if (c == kFirst && MODE != kModeScores) cp_async_wait_all();
+#pragma unroll 1
+        for (int i = 0; i < per && jn < nn; ++i, jn += NT) keys[jn] = sc_key_from<MODE>(p, gn, jn, keys[jn]);
+      }
+      __syncthreads();  // every load of the chunk has landed before any store
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int q = base + u * rows_per_pass + my_row;
+        if (active && q < M) {
+          const int64_t drow = sc_row(p, g, P + q);
+          *reinterpret_cast<uint4 *>(p.k_pool + drow * rb + my_vec * 16) = kr[u];
+          *reinterpret_cast<uint4 *>(p.v_pool + drow * rb + my_vec * 16) = vr[u];
+          if (my_vec == 0) p.pos_map[drow] = pr[u];
+        }
+      }
+    }
+    if (tid == 0 && M > q0) atomicAdd(p.counters, (unsigned long long)(M - q0));
+    if (!more) break;
+    // copies that the loop was too short to cover
+    if (MODE != kModeScores && nchunks < 2) {
+      if (nchunks == 0) {
+        cp_async_wait_all();
+        __syncthreads();  // the row is visible
+      }
+      fetch_positions();
+    }
+    cp_async_wait_all();
+    for (; jn < nn; jn += NT) keys[jn] = sc_key_from<MODE>(p, gn, jn, keys[jn]);
+    g = gn;
+    buf ^= 1;
+  }
+}
+
 template <int NT, int U, int MODE, int VAR>
 cudaError_t launch_one(const SelectCompactParams &p, int n_seg_req, int keys_cap, size_t smem,
                        cudaStream_t s) {
@@ -429,12 +665,52 @@ cudaError_t launch_one(const SelectCompactParams &p, int n_seg_req, int keys_cap
   return cudaGetLastError();
 }
 
+// Shared memory of the persistent form: keys, the rank map (sized by the
+// launch's largest M) and two block-table rows.
+inline size_t pipe_smem(const SelectCompactParams &p, int keys_cap, int m_cap) {
+  return (size_t)keys_cap * sizeof(uint32_t) + (size_t)m_cap * sizeof(uint16_t) +
+         (size_t)2 * p.bt_stride * sizeof(int32_t);
+}
+// The copy's loads in flight are staged in L1, which shares its storage with
+// shared memory: past the 196 KB carve-out (this much dynamic shared memory,
+// plus the static scratch and the 1 KB the runtime reserves per CTA) only
+// 28 KB of L1 remain and the copy slows by about 15 % against the 60 KB that
+// 196 KB leaves (measured), so larger launches take the one-CTA-per-segment
+// kernel instead.
+constexpr size_t kPipeSmemMax = 192 * 1024;
+
+template <int MODE, int VAR>
+cudaError_t launch_pipe(const SelectCompactParams &p, int n_seg_req, int keys_cap, int m_cap, cudaStream_t s) {
+  auto kernel = select_compact_pipe_kernel<MODE, KVC_SC_UNROLL_LARGE, VAR>;
+  const size_t smem = pipe_smem(p, keys_cap, m_cap);
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148, per_sm = 1;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 512, smem)) != cudaSuccess) return e;
+  const int n_items = n_seg_req * p.layers * p.hkv;
+  const int grid = std::min(n_items, sms * std::max(per_sm, 1));
+  if ((e = cudaMemsetAsync(sc_work_counter(p), 0, sizeof(int), s)) != cudaSuccess) return e;
+  kernel<<<grid, 512, smem, s>>>(p, n_items, keys_cap, m_cap);
+  return cudaGetLastError();
+}
+
 template <int NT, int U, int MODE>
-cudaError_t launch_var(const SelectCompactParams &p, int var, int n_seg_req, int keys_cap, size_t smem,
-                       cudaStream_t s) {
+cudaError_t launch_var(const SelectCompactParams &p, int var, int n_seg_req, int keys_cap, int m_cap,
+                       size_t smem, cudaStream_t s) {
+  // order-preserving rounds with more than 4096 candidates: the persistent
+  // form where its shared memory leaves the copy enough L1
+  const bool pipe = NT == 512 && pipe_smem(p, keys_cap, m_cap) <= kPipeSmemMax;
   switch (var) {
-    case kOrderedSlotTie: return launch_one<NT, U, MODE, kOrderedSlotTie>(p, n_seg_req, keys_cap, smem, s);
-    case kOrderedPosTie: return launch_one<NT, U, MODE, kOrderedPosTie>(p, n_seg_req, keys_cap, smem, s);
+    case kOrderedSlotTie:
+      if constexpr (NT == 512)
+        if (pipe) return launch_pipe<MODE, kOrderedSlotTie>(p, n_seg_req, keys_cap, m_cap, s);
+      return launch_one<NT, U, MODE, kOrderedSlotTie>(p, n_seg_req, keys_cap, smem, s);
+    case kOrderedPosTie:
+      if constexpr (NT == 512)
+        if (pipe) return launch_pipe<MODE, kOrderedPosTie>(p, n_seg_req, keys_cap, m_cap, s);
+      return launch_one<NT, U, MODE, kOrderedPosTie>(p, n_seg_req, keys_cap, smem, s);
     // hole filling moves few rows: a short copy chunk keeps registers low and
     // lets more CTAs per SM hide the latency of the select phase
     default: return launch_one<NT, KVC_SC_UNROLL_HOLE, MODE, kHoleFill>(p, n_seg_req, keys_cap, smem, s);
@@ -442,14 +718,16 @@ cudaError_t launch_var(const SelectCompactParams &p, int var, int n_seg_req, int
 }
 
 template <int NT, int U>
-cudaError_t launch_nt(const SelectCompactParams &p, int mode, int var, int n_seg_req, int max_n,
+cudaError_t launch_nt(const SelectCompactParams &p, int mode, int var, int n_seg_req, int max_n, int max_m,
                       cudaStream_t s) {
   const int keys_cap = (max_n + 7) & ~7;
+  const int m_cap = (max_m + 7) & ~7;
   const size_t smem = (size_t)keys_cap * (sizeof(uint32_t) + sizeof(uint16_t));
   switch (mode) {
-    case kModeRandom: return launch_var<NT, U, kModeRandom>(p, var, n_seg_req, keys_cap, smem, s);
-    case kModeRandomShared: return launch_var<NT, U, kModeRandomShared>(p, var, n_seg_req, keys_cap, smem, s);
-    default: return launch_var<NT, U, kModeScores>(p, var, n_seg_req, keys_cap, smem, s);
+    case kModeRandom: return launch_var<NT, U, kModeRandom>(p, var, n_seg_req, keys_cap, m_cap, smem, s);
+    case kModeRandomShared:
+      return launch_var<NT, U, kModeRandomShared>(p, var, n_seg_req, keys_cap, m_cap, smem, s);
+    default: return launch_var<NT, U, kModeScores>(p, var, n_seg_req, keys_cap, m_cap, smem, s);
   }
 }
 
@@ -457,11 +735,11 @@ cudaError_t launch_nt(const SelectCompactParams &p, int mode, int var, int n_seg
 
 cudaError_t launch_select_compact(const SelectCompactParams &p, int mode, int n_seg_req,
                                   int max_n, int max_m, cudaStream_t s) {
-  (void)max_m;
   if (n_seg_req <= 0) return cudaSuccess;
   const int var = (p.flags & kScHoleFill) ? kHoleFill : (p.flags & kScTieByPos) ? kOrderedPosTie : kOrderedSlotTie;
-  if (max_n <= KVC_SC_NT256_MAX_N) return launch_nt<256, KVC_SC_UNROLL_SMALL>(p, mode, var, n_seg_req, max_n, s);
-  return launch_nt<512, KVC_SC_UNROLL_LARGE>(p, mode, var, n_seg_req, max_n, s);
+  if (max_n <= KVC_SC_NT256_MAX_N)
+    return launch_nt<256, KVC_SC_UNROLL_SMALL>(p, mode, var, n_seg_req, max_n, max_m, s);
+  return launch_nt<512, KVC_SC_UNROLL_LARGE>(p, mode, var, n_seg_req, max_n, max_m, s);
 }
 
 }  // namespace kvc
