@@ -219,6 +219,18 @@ def test_long_trace_every_request():
     print(out)
 
 
+def test_large_survivor_count():
+    """Beacon selection on segments of 32768 and 9000 keys keeping most of them: the rank map is too large for the
+    persistent select form's shared memory budget, so the round takes the one-CTA-per-segment kernel."""
+    P = np.array([0, 100])
+    L = np.array([32768, 9000])
+    K = np.array([30000, 8000])
+    w = wl.Workload("large_m_beacon", 2, 1, 2, 128, P, L, K, selectors=("beacon",), num_q_heads=8,
+                    num_beacons=64, query_window=64, n_components=64, data_seed=47, philox_seed=53)
+    out = run_beacon(w)
+    print(out)
+
+
 def _sharp(w):
     return wl.scaled(w, query_norm=math.sqrt(w.head_dim))
 

@@ -156,3 +156,16 @@ def test_ragged_sweep_slice(c, sel):
     the K/V bytes of one layer and a sample of the 32-bit draws."""
     w = wl.scaled(wl.ragged(c), num_layers=12, num_beacons=0, query_window=0, num_q_heads=8)
     run_rounds(w, sel, rounds=1, seed=w.philox_seed, kv_layers=[5], check_scores_n=500)
+
+
+@pytest.mark.parametrize("selector", ["random", "random_shared"])
+def test_large_survivor_counts(selector):
+    """Segments of up to 32768 candidates that keep most of them: the rank map is too large for the persistent
+    form's shared memory budget, so the round takes the one-CTA-per-segment kernel (two rounds)."""
+    cases = [(0, 32768, 30000), (100, 20000, 19000), (50, 5000, 4000), (7, 4133, 1000)]
+    P = np.array([c[0] for c in cases])
+    L = np.array([c[1] for c in cases])
+    K = np.array([c[2] for c in cases])
+    w = wl.Workload("large_m", len(cases), 1, 2, 128, P, L, K, selectors=(selector,), trigger=40,
+                    data_seed=41, philox_seed=43)
+    run_rounds(w, selector, rounds=2, seed=w.philox_seed, check_scores_n=400)

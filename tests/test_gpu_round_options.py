@@ -123,6 +123,14 @@ def test_block_draws(block, selector):
     run_option_rounds(_workload(), selector, [{"block": block}, {"block": block}], seed=11)
 
 
+@pytest.mark.parametrize("selector", ["random", "random_shared"])
+def test_block_draws_as_long_as_the_segment(selector):
+    """One draw for a whole segment (block 32768: every candidate ties and the lowest slots stay, so no row
+    moves) and two draws for the 4133-slot request (block 4096: a few dozen rows move): the persistent select
+    form's rounds whose copy is empty or a single chunk."""
+    run_option_rounds(_workload(), selector, [{"block": 32768}, {"block": 4096}, {}], seed=13)
+
+
 def test_block_one_equals_default():
     w = _workload(layers=1, H=2)
     run_option_rounds(w, "random", [{"block": 1}, {}], seed=3)
