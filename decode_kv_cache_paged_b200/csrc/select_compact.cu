@@ -73,24 +73,28 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
 // the bucket holding the answer has at most kFinish keys (for random 32-bit
 // keys that is after the first digit), those keys are gathered and one warp
 // finishes by counting, so the remaining passes over all keys are skipped.
+// first_ready: hist already holds the top-byte counts of every key (built
+// while the keys were drawn), so the first digit needs no pass.
 constexpr int kFinish = 64;
 
 template <int NT, class KeyFn>
 __device__ __forceinline__ void block_radix_select(int n, int k_in, KeyFn keyfn, uint32_t *hist,
                                                    uint32_t *bcast, uint32_t *cand, uint32_t &tau,
-                                                   int &need, int &count_eq) {
+                                                   int &need, int &count_eq, bool first_ready = false) {
   uint32_t prefix = 0, mask = 0;
   int k = k_in;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 #pragma unroll 1
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += NT) hist[i] = 0;
-    __syncthreads();
-    for (int j = tid; j < n; j += NT) {
-      uint32_t key;
-      if (keyfn(j, key) && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    if (!(first_ready && shift == 24)) {
+      for (int i = tid; i < 256; i += NT) hist[i] = 0;
+      __syncthreads();
+      for (int j = tid; j < n; j += NT) {
+        uint32_t key;
+        if (keyfn(j, key) && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
     }
-    __syncthreads();
     if (warp == 0) {
       // lane l owns digits 255-8l .. 248-8l (descending)
       uint32_t c[8];
@@ -278,11 +282,12 @@ struct ScThreshold {
 
 template <int NT, int VAR>
 __device__ __forceinline__ ScThreshold sc_threshold(const SelectCompactParams &p, const ScSeg &g,
-                                                    const uint32_t *keys, ScScratch<NT> &sh) {
+                                                    const uint32_t *keys, ScScratch<NT> &sh,
+                                                    bool hist_ready = false) {
   ScThreshold t;
   block_radix_select<NT>(
       g.N, g.M, [&](int j, uint32_t &k) { k = keys[j]; return true; }, sh.hist, sh.bcast, sh.cand, t.tau, t.need,
-      t.count_eq);
+      t.count_eq, hist_ready);
   // with ties split and slots possibly out of position order: the `need`
   // lowest positions among the tied keys (positions are distinct)
   t.ptau = 0;
@@ -520,7 +525,8 @@ __host__ __device__ __forceinline__ int *sc_work_counter(const SelectCompactPara
 //     position of every candidate (random selectors) into the keys buffer;
 //   - from the next chunk on, between issuing the chunk's loads and its
 //     barrier, each thread turns a share of the words it fetched itself into
-//     keys (Philox draws, or the scores' order keys).
+//     keys (Philox draws, or the scores' order keys) and counts their top
+//     bytes, so the threshold's first radix digit needs no pass of its own.
 // No dependent global load sits between a chunk's loads and its stores, so
 // the draws never wait behind the copy's loads in flight.  The keys buffer is
 // free during the copy (the copy reads only src_of_rank), and the next
@@ -550,9 +556,14 @@ __global__ void __launch_bounds__(512, 1)
   {
     const int pages = (g.P + g.N + kPage - 1) / kPage;
     for (int i = tid; i < pages; i += NT) bt_buf[i] = g.bt[i];
+    for (int i = tid; i < 256; i += NT) sh.hist[i] = 0;
     g.bt = bt_buf;
     __syncthreads();
-    for (int j = tid; j < g.N; j += NT) keys[j] = sc_key<MODE>(p, g, j);
+    for (int j = tid; j < g.N; j += NT) {
+      const uint32_t key = sc_key<MODE>(p, g, j);
+      keys[j] = key;
+      atomicAdd(&sh.hist[key >> 24], 1u);
+    }
   }
 
   const int vpr = p.row_bytes >> 4;  // 16-byte vectors per row
@@ -566,12 +577,14 @@ __global__ void __launch_bounds__(512, 1)
   while (true) {
     if (tid == 0) sh.first_evicted = g.N;
     __syncthreads();  // the keys of g are complete
-    const ScThreshold t = sc_threshold<NT, VAR>(p, g, keys, sh);
+    const ScThreshold t = sc_threshold<NT, VAR>(p, g, keys, sh, true);
     sc_ordered_ranks<NT, VAR>(p, g, keys, t, src_of_rank, sh);
     const int q0 = sh.first_evicted;
     // the next item; every thread has read sh.next of the previous one and
-    // sh.first_evicted of this one before the barrier
+    // sh.first_evicted of this one before the barrier.  The histogram is
+    // free again: the next segment's draws count their top bytes into it
     if (tid == 0) sh.next = atomicAdd(work, 1);
+    for (int i = tid; i < 256; i += NT) sh.hist[i] = 0;
     __syncthreads();
     const int nxt = sh.next;
     const bool more = nxt < n_items;
@@ -623,7 +636,11 @@ __global__ void __launch_bounds__(512, 1)
       if (c >= kFirst) {
         if (c == kFirst && MODE != kModeScores) cp_async_wait_all();
 #pragma unroll 1
-        for (int i = 0; i < per && jn < nn; ++i, jn += NT) keys[jn] = sc_key_from<MODE>(p, gn, jn, keys[jn]);
+        for (int i = 0; i < per && jn < nn; ++i, jn += NT) {
+          const uint32_t key = sc_key_from<MODE>(p, gn, jn, keys[jn]);
+          keys[jn] = key;
+          atomicAdd(&sh.hist[key >> 24], 1u);
+        }
       }
       __syncthreads();  // every load of the chunk has landed before any store
 #pragma unroll
@@ -648,7 +665,11 @@ __global__ void __launch_bounds__(512, 1)
       fetch_positions();
     }
     cp_async_wait_all();
-    for (; jn < nn; jn += NT) keys[jn] = sc_key_from<MODE>(p, gn, jn, keys[jn]);
+    for (; jn < nn; jn += NT) {
+      const uint32_t key = sc_key_from<MODE>(p, gn, jn, keys[jn]);
+      keys[jn] = key;
+      atomicAdd(&sh.hist[key >> 24], 1u);
+    }
     g = gn;
     buf ^= 1;
   }
